@@ -1,0 +1,444 @@
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one attention layer over the whole batch of the
+Llama-3-8B-shaped GQA workload (256 sequences, 32 query / 8 KV heads,
+head_dim 128, block 16, bf16 cache, log-normal lengths with median 1024
+clipped to [16, 8192]): copy-on-write copies, append of one new token per
+sequence, and split-context attention (512-token partitions + merge).
+
+``value``: KV GB/s = algorithmic K/V bytes of a step (every (token, KV head)
+row of K and V once) / device time of a step, inputs resident in HBM, the same
+decode step repeated (appends rewrite the same slots, so the workload stays
+the stated one).  The K/V set (1.7 GB) is far larger than L2 (126 MB), so no
+flush is needed between steps.  ``e2e``: the same metric through the public
+API from pinned host buffers: every step reserves its slots on the host,
+copies q / new K,V / slots / tables to the device, runs the kernels and reads
+the output back (sequences grow by one token per step there).
+
+``--impl reference`` times the CPU oracle (float64 numpy) on a bounded sample
+of the same workload.  Under torchrun every rank runs its own replica of the
+batch (weak scaling); rank 0 prints the JSON line with the max time over ranks.
+"""
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; decode tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_gqa")
+    ap.add_argument("--partition", type=int, default=None, help="override the workload's partition size")
+    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def traffic_record(workload):
+    """dram bytes per decode launch from a committed ncu summary, if it matches the current kernel source."""
+    from paged_kv_cache_341_b200 import build
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = build.kernel_digest()
+    entry = rec.get(workload)
+    if not entry or entry.get("kernel_digest") != src:
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(sc, seqs, q_host):
+    """Time the oracle on sequences ``seqs`` of the scenario's batch; returns (seconds, kv bytes)."""
+    from oracle import oracle_decode
+
+    class F64:
+        def __init__(self, t):
+            self.t, self.shape = t, tuple(t.shape)
+
+        def __getitem__(self, i):
+            return self.t[i].to(torch.float64).numpy()
+
+    w, c = sc.w, sc.cache
+    rows = list(range(sc.rows.start, sc.rows.stop))
+    tables = [list(c.tables[r]) for r in rows]
+    lens = [int(c.lens[r]) for r in rows]
+    qd = q_host.double().numpy()
+    t0 = time.perf_counter()
+    oracle_decode(qd, F64(sc.k_host), F64(sc.v_host), tables, lens, w.scale, seqs=seqs)
+    dt = time.perf_counter() - t0
+    nbytes = sum(lens[s] for s in seqs) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+    return dt, nbytes
+
+
+def pick_sample(sc, budget_s, q_host):
+    """Sequences (round-robin over the batch) whose oracle time fits ``budget_s``."""
+    dt, _ = oracle_sample(sc, [0], q_host)
+    per_seq = max(dt, 1e-4)
+    n = int(max(1, min(sc.batch, budget_s / per_seq)))
+    return list(range(0, sc.batch, max(1, sc.batch // n)))[:n]
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    sc = ReferenceScenario(args.workload)
+    q_host, _, _ = sc.step_inputs(0)
+    per_step_budget = max(0.002, 90.0 / (args.steps + args.warmup))
+    seqs = pick_sample(sc, per_step_budget, q_host)
+    for _ in range(args.warmup):
+        oracle_sample(sc, seqs, q_host)
+    total_t, total_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = oracle_sample(sc, seqs, q_host)
+        total_t += dt
+        total_b += nb
+    gbs = total_b / total_t / 1e9
+    cores = cpu_threads()
+    sample = "%d of %d sequences per step (%d tokens), oracle float64 numpy" % (
+        len(seqs), sc.batch, sum(int(sc.cache.lens[sc.rows.start + s]) for s in seqs))
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_t / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(sc, args),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+class ReferenceScenario:
+    """The workload on the host only (no GPU): tables from the oracle pool, values from the generator."""
+
+    def __init__(self, name):
+        from oracle import OraclePool
+        from paged_kv_cache_341_b200 import workloads
+        w = workloads.get(name)
+        self.w = w
+        self.lens0 = workloads.lengths(w)
+        op = OraclePool(w.num_blocks, w.block_size, workloads.pool_order(w.num_blocks, w.seed))
+        s = w.num_seqs
+        rows = 2 * s if w.shared_prefix else s
+        tables = np.full((rows, w.max_blocks_per_seq), -1, np.int32)
+        lens = np.zeros(rows, np.int32)
+        if w.shared_prefix:
+            prefix = op.alloc(w.shared_prefix // w.block_size)
+            for r in range(s):
+                if r:
+                    op.fork(prefix)
+                ids = prefix + op.alloc(-(-int(self.lens0[r]) // w.block_size))
+                tables[r, :len(ids)] = ids
+                lens[r] = w.shared_prefix + int(self.lens0[r])
+            for r in range(s):
+                n = -(-int(lens[r]) // w.block_size)
+                op.fork(list(tables[r, :n]))
+                tables[s + r], lens[s + r] = tables[r], lens[r]
+            self.rows = slice(s, 2 * s)
+        else:
+            for r in range(s):
+                ids = op.alloc(-(-int(self.lens0[r]) // w.block_size))
+                tables[r, :len(ids)] = ids
+                lens[r] = int(self.lens0[r])
+            self.rows = slice(0, s)
+        self.cache = type("HostTables", (), {"tables": tables, "lens": lens})()
+        used = sorted({int(b) for r in range(rows) for b in tables[r, :-(-int(lens[r]) // w.block_size)]})
+        self.k_host, self.v_host = workloads.fill_blocks(w, used, w.seed + 100)
+
+    @property
+    def batch(self):
+        return self.rows.stop - self.rows.start
+
+    def step_inputs(self, step):
+        from paged_kv_cache_341_b200 import workloads
+        seed = self.w.seed + 1000 + 10 * step
+        return workloads.queries(self.w, seed, num_seqs=self.batch), None, None
+
+
+def workload_config(sc, args):
+    w = sc.w
+    lens = sc.cache.lens[sc.rows.start:sc.rows.stop]
+    p = w.partition_size if args.partition is None else args.partition
+    return {"workload": w.name, "num_seqs": int(sc.batch), "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "cache_dtype": w.dtype,
+            "mean_context": round(float(np.mean(lens)), 1), "max_context": int(np.max(lens)),
+            "partition_size": p, "num_blocks": w.num_blocks, "layers": 1,
+            "l2": "inputs larger than L2 (K/V set %.2f GB vs 126 MB L2), no flush" % (
+                int(np.sum(lens)) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes / 1e9),
+            "parallelism": "replicas x%d (weak)" % args.gpus}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from paged_kv_cache_341_b200 import build, pa
+    build.ensure_built()
+    from paged_kv_cache_341_b200.scenarios import Scenario
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    sc = Scenario(args.workload, keep_host=want_cpu)
+    w, c = sc.w, sc.cache
+    part = w.partition_size if args.partition is None else args.partition
+    stream = torch.cuda.current_stream()
+
+    # ---- one stationary decode step, inputs resident in HBM
+    q_h, kn_h, vn_h = sc.step_inputs(0)
+    q, kn, vn = q_h.cuda(), kn_h.cuda(), vn_h.cuda()
+    slots, pairs = c.reserve(sc.rows)
+    c.upload_tables()
+    d_slots = torch.from_numpy(slots).cuda()
+    d_pairs = torch.from_numpy(np.ascontiguousarray(pairs)).cuda()
+    tables = c.d_tables[sc.rows]
+    lens = c.d_lens[sc.rows]
+    out = torch.empty((sc.batch, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device="cuda")
+    ws = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
+    kv_bytes = sc.kv_bytes()
+    launches_per_step = (1 if pairs.shape[0] else 0) + 1 + (2 if part > 0 else 1)
+
+    def step(ev0=None, ev1=None):
+        c.copy_blocks(d_pairs)
+        c.append(kn, vn, d_slots)
+        if ev0 is not None:
+            ev0.record(stream)
+        c.attend(q, out, w.scale, part, ws, tables=tables, lens=lens)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_att = min(args.steps, 256)
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_att)]
+    t_start.record(stream)
+    for i in range(args.steps):
+        if i < n_att:
+            step(*att_ev[i])
+        else:
+            step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = t_start.elapsed_time(t_end) / args.steps
+    att_ms = float(np.mean([a.elapsed_time(b) for a, b in att_ev]))
+    if world > 1:
+        t = torch.tensor([ms, att_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, att_ms = float(t[0]), float(t[1])
+    assert pa.pa_device_error() == 0
+
+    # ---- end to end through the public API from pinned host memory
+    e2e = None
+    if args.e2e_steps > 0:
+        n_e2e = args.e2e_steps
+        host_in = []
+        for i in range(n_e2e):
+            qi, ki, vi = sc.step_inputs(1 + i)
+            host_in.append((qi.pin_memory(), ki.pin_memory(), vi.pin_memory()))
+        q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        in_bytes = q.numel() * q.element_size() + 2 * kn.numel() * kn.element_size()
+        meta_bytes = (c.d_tables.numel() + c.d_lens.numel()) * 4 + sc.batch * 8
+        e2e_bytes, pairs_total = 0, 0
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_e2e):
+            qi, ki, vi = host_in[i]
+            q_d.copy_(qi, non_blocking=True)
+            k_d.copy_(ki, non_blocking=True)
+            v_d.copy_(vi, non_blocking=True)
+            _, pr = c.decode_step(q_d, k_d, v_d, out, w.scale, part, ws_e2e(pa, sc, part), rows=sc.rows)
+            pairs_total += pr.shape[0]
+            out_h.copy_(out, non_blocking=True)
+            stream.synchronize()
+            e2e_bytes += sc.kv_bytes()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        e2e = {"value": round(world * e2e_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(in_bytes + meta_bytes + 8 * pairs_total / max(1, n_e2e)),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()), "steps": n_e2e,
+               "ms_per_step": round(e2e_ms / n_e2e, 4),
+               "note": "host slot reservation, pinned H2D of q/new K,V/slots/tables, kernels, D2H of out; "
+                       "sequences grow one token per step"}
+        assert pa.pa_device_error() == 0
+
+    # ---- CPU oracle baseline on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if want_cpu:
+        seqs = pick_sample(sc, 15.0, q_h)
+        dt, nb = oracle_sample(sc, seqs, q_h)
+        cpu = {"value": round(nb / dt / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": "%d of %d sequences of one step (%d tokens), float64 numpy, %.1f s" % (
+                   len(seqs), sc.batch, sum(int(c.lens[sc.rows.start + s]) for s in seqs), dt),
+               "host_cpus": os.cpu_count()}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        value = world * kv_bytes / (ms / 1e3) / 1e9
+        achieved = kv_bytes / (att_ms / 1e3) / 1e9
+        traffic = traffic_record(w.name)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": workload_config(sc, args),
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "pct_of_8tbs_spec": round(100 * value / world / 8000.0, 2),
+            "decode_tokens_per_s": round(world * sc.batch / (ms / 1e3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "kernel": "pa_decode_attention (decode_kernel + reduce_kernel), mean of %d launches; "
+                                   "peak = %s copy bandwidth" % (n_att, peak_kind),
+                         "algorithmic_bytes_per_launch": kv_bytes},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+_WS = {}
+
+
+def ws_e2e(pa, sc, part):
+    key = id(sc)
+    if key not in _WS:
+        w, c = sc.w, sc.cache
+        _WS[key] = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
+    return _WS[key]
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * pa.h -- C ABI of libpagedattn.so, a paged KV cache decode path for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What it implements, from the descriptions of PagedAttention on four web
+ * pages (no code from them is used):
+ *
+ *   - a pool of equally sized physical KV blocks that each sequence reaches
+ *     through its own block table ("PagedAttention Explained: Managing KV Cache
+ *     Efficiently", agentechip.com, section "Block Tables and Non-Contiguous
+ *     Storage"; "Master Paged Attention for LLM Inference", krapton.com,
+ *     section "How Paged Attention Works: The Mechanics", steps 1-3);
+ *   - blocks handed out on demand from a first-in first-out free list, with a
+ *     reference count per block, and copy-on-write for blocks that several
+ *     sequences share (agentechip.com, sections "Implementing a Simplified
+ *     Paged KV Cache" and "Shared Prefix Caching"; krapton.com step 4);
+ *   - the device kernels of one decode step: copy of shared blocks before a
+ *     write, append of the new token's K/V into its slot, and single-query
+ *     attention that walks the block table instead of gathering the blocks
+ *     (agentechip.com, "Block Tables and Non-Contiguous Storage" and the
+ *     closing remark of "Implementing a Simplified Paged KV Cache").
+ *
+ * Conventions for every call:
+ *   - Status codes only; nothing throws, aborts or traps.  On failure,
+ *     pa_last_error() returns a message (per calling thread).
+ *   - The library allocates NO device memory.  Caches, tables, workspace and
+ *     outputs are device buffers owned by the caller (e.g. torch tensors'
+ *     data_ptr()).  Host arrays are owned by the caller too.
+ *   - Device calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and only enqueue work.  A launch failure returns
+ *     PA_ERR_CUDA.  Bad indices found on the device (a block id outside the
+ *     pool, a slot outside the cache, a length beyond the table) never fault:
+ *     the access is skipped or clamped and a device error word is set, which
+ *     pa_device_error() reads after the stream is synchronised.
+ *   - Cache layout, K and V alike: [num_blocks][block_size][num_kv_heads]
+ *     [head_dim], contiguous, element type `dtype` -- each block holds
+ *     block_size token rows of (num_kv_heads, head_dim), the per-block shape of
+ *     the toy cache in agentechip.com "Implementing a Simplified Paged KV
+ *     Cache".  Device pointers must be 16-byte aligned.
+ *   - A flat slot index x names block x / block_size, row x % block_size.
+ */
+#ifndef PAGEDATTN_PA_H
+#define PAGEDATTN_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_EXHAUSTED = 1,     /* no free block: the pages' "KV cache exhausted"   */
+  PA_ERR_INVALID = 2,       /* bad argument (range, size, alignment, null)      */
+  PA_ERR_REFCOUNT = 3,      /* release/share not allowed by the reference count */
+  PA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed             */
+  PA_ERR_DEVICE_CHECK = 5,  /* a kernel found a bad index (see pa_device_error) */
+  PA_ERR_UNSUPPORTED = 6    /* shape/dtype combination not compiled in          */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* ------------------------------------------------------------------------ */
+/* Host block pool.  Opaque, host memory only, not thread-safe.             */
+/* Every failing call leaves the pool unchanged (all or nothing).           */
+/* ------------------------------------------------------------------------ */
+typedef struct pa_pool pa_pool;
+
+/* Create a pool of `num_blocks` blocks of `block_size` tokens.  The free list
+ * starts as `initial_free_order` (a permutation of 0..num_blocks-1, copied),
+ * or as 0..num_blocks-1 when it is NULL (the toy pool's starting list in
+ * agentechip.com "Implementing a Simplified Paged KV Cache").
+ * Errors: PA_ERR_INVALID (num_blocks < 0, block_size <= 0, not a permutation,
+ * out == NULL). */
+pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
+                         const int32_t* initial_free_order, pa_pool** out);
+void pa_pool_destroy(pa_pool* pool);
+
+/* Take `n` blocks from the FRONT of the free list into out_ids[0..n), each
+ * with reference count 1.  Errors: PA_ERR_EXHAUSTED if fewer than n are
+ * free; PA_ERR_INVALID for n < 0 or a NULL buffer with n > 0. */
+pa_status pa_pool_alloc(pa_pool* pool, int32_t n, int32_t* out_ids);
+
+/* Drop one reference per listed id (duplicates count twice); a block whose
+ * count reaches 0 goes to the BACK of the free list, in list order
+ * (agentechip.com "Implementing a Simplified Paged KV Cache").  Errors:
+ * PA_ERR_INVALID (id out of range), PA_ERR_REFCOUNT (more releases than
+ * references). */
+pa_status pa_pool_free(pa_pool* pool, const int32_t* ids, int32_t n);
+
+/* Add one reference per listed id: a second sequence now shares the block
+ * (copy-on-write sharing, krapton.com step 4 "Shared Blocks").  The caller
+ * copies the parent's table and length for the child.  Errors:
+ * PA_ERR_INVALID (id out of range), PA_ERR_REFCOUNT (block is free). */
+pa_status pa_pool_fork(pa_pool* pool, const int32_t* ids, int32_t n);
+
+pa_status pa_pool_refcount(const pa_pool* pool, int32_t id, int32_t* out);
+pa_status pa_pool_num_free(const pa_pool* pool, int32_t* out);
+
+/* Copy the state out: refcounts[num_blocks] by block id, free_list[n_free]
+ * front to back (buffer of num_blocks entries). */
+pa_status pa_pool_export(const pa_pool* pool, int32_t* refcounts, int32_t* free_list,
+                         int32_t* n_free);
+
+/* Reserve the slot of token number *len of one sequence and advance *len.
+ * `table` is the sequence's host block table with room for `table_cap`
+ * entries.  Offset 0 of a block takes a fresh block from the free list.  At
+ * offset > 0, when the current block's count is above 1 (shared), the
+ * sequence moves to a fresh block: the old block loses one reference, the
+ * table entry changes, and (*cow_src_out, *cow_dst_out) name the copy the
+ * caller must run (pa_copy_blocks) before appending; otherwise both are -1.
+ * The plainest reading of "copy-on-write" on the pages (agentechip.com
+ * "Shared Prefix Caching"), which give no trigger rule of their own.
+ * Errors: PA_ERR_EXHAUSTED (no block for a new block or a copy),
+ * PA_ERR_INVALID (table too small, table entry free or out of range). */
+pa_status pa_seq_reserve_slot(pa_pool* pool, int32_t* table, int32_t table_cap, int32_t* len,
+                              int64_t* slot_out, int32_t* cow_src_out, int32_t* cow_dst_out);
+
+/* One decode step's reservations for S sequences, in order s = 0..S-1:
+ * pa_seq_reserve_slot on row s of `tables` ([S][table_cap], host) with
+ * lens[s]; slots_out[s] receives the slot; every copy-on-write pair is
+ * appended to pairs_out ([S][2] room) and counted in *num_pairs_out.  All or
+ * nothing: on any failure the pool, tables and lens are restored. */
+pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, int32_t* lens,
+                           int32_t num_seqs, int64_t* slots_out, int32_t* pairs_out,
+                           int32_t* num_pairs_out);
+
+/* ------------------------------------------------------------------------ */
+/* Device kernels (sm_100a).                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Append: for t < T with slot_mapping[t] >= 0, write k_new[t] ([Hkv][D]) and
+ * v_new[t] into row slot % block_size of block slot / block_size (the write of
+ * a new token into its block, agentechip.com "Implementing a Simplified Paged
+ * KV Cache").  k_new, v_new: device [T][Hkv][D]; slot_mapping: device int64
+ * [T]; slots must be distinct.  A slot >= num_blocks*block_size is skipped and
+ * sets the device error word.  Bit copy. */
+pa_status pa_append_kv(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                       int32_t num_tokens, void* k_cache, void* v_cache, int32_t num_blocks,
+                       int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                       pa_dtype dtype, void* stream);
+
+/* Copy-on-write block copy: for each pair p, K and V block pairs[p][1] become
+ * bit copies of block pairs[p][0] (krapton.com step 4; agentechip.com
+ * "Shared Prefix Caching").  pairs: device int32 [P][2]; destinations must be
+ * distinct and no destination may also be a source in the same call.  Ids
+ * outside [0, num_blocks) are skipped and set the device error word. */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_pairs,
+                         int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                         int32_t head_dim, pa_dtype dtype, void* stream);
+
+/* Bytes of device workspace pa_decode_attention needs for these sizes: 0 when
+ * partition_size == 0, else room for one float32 partial (max, sum, D values)
+ * per (sequence, query head, partition), partitions = ceil(max_blocks_per_seq
+ * * block_size / partition_size). */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_blocks_per_seq, int32_t block_size,
+                                int32_t partition_size);
+
+/* Single-query decode attention over the paged cache.  For every sequence s
+ * and query head h, with kv = h / (Hq / Hkv):
+ *   out[s][h] = softmax_j(q[s][h] . K_s[j][kv] * scale) V_s[j][kv],
+ *   j < context_lens[s], where K_s[j] is row j % block_size of block
+ *   block_tables[s][j / block_size] (and V likewise).
+ * That is ordinary attention over the sequence's tokens in logical order: the
+ * kernel walks the block table and never gathers the blocks
+ * (agentechip.com "Block Tables and Non-Contiguous Storage"; krapton.com
+ * "FAQ": paging leaves the computation unchanged).  Accumulation is float32
+ * (online softmax with a running maximum and sum).  Grouped query heads
+ * (Hq > Hkv) share every K/V load.  context_lens[s] == 0 writes a zero row.
+ *
+ *   q, out:        device [S][Hq][D], element type dtype (out rounded to
+ *                  nearest even from float32)
+ *   k/v_cache:     device [num_blocks][block_size][Hkv][D]
+ *   block_tables:  device int32 [S][max_blocks_per_seq]; entries that cover
+ *                  tokens < context_lens[s] must be valid block ids
+ *   context_lens:  device int32 [S], each <= max_blocks_per_seq*block_size
+ *   partition_size 0: one pass over each whole context.  > 0 (a multiple of
+ *                  block_size): split each context into partitions of
+ *                  that many tokens, compute partial (max, sum, output) per
+ *                  partition and merge them with a second kernel; needs
+ *                  `workspace` of pa_decode_workspace_size() bytes.
+ * Supported: head_dim 64 or 128; Hq/Hkv in {1,2,4,8}; block_size a multiple
+ * of 16; dtype f32/f16/bf16.  Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED,
+ * PA_ERR_CUDA. */
+pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_cache,
+                              int32_t num_blocks, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, float scale,
+                              int32_t partition_size, void* workspace, size_t workspace_bytes,
+                              void* out, pa_dtype dtype, void* stream);
+
+/* Read (and, if reset != 0, clear) the device error word of the current
+ * device: 0 = none; 1 = block id outside the pool in a table; 2 =
+ * context length beyond the table; 3 = append slot outside the cache; 4 =
+ * copy pair id outside the pool.  Synchronous: waits for the device. */
+pa_status pa_device_error(int32_t* code_out, int32_t reset);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_PA_H */

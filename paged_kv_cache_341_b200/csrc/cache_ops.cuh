@@ -1,0 +1,57 @@
+// Cache-maintenance kernels of one decode step (bit copies, HBM-bound).
+//
+// append_kernel: the new token's K/V row goes into its slot -- the write of a
+//   token into the next position of its block ("PagedAttention Explained:
+//   Managing KV Cache Efficiently", section "Implementing a Simplified Paged KV
+//   Cache").  A cache row [Hkv][D] is contiguous and flat row index == slot, so
+//   one CTA copies one row with 16-byte vector loads/stores.
+// copy_kernel: copy-on-write of a shared block before a sequence writes into
+//   it (krapton.com "How Paged Attention Works", step 4; agentechip.com "Shared
+//   Prefix Caching").  A block is block_size contiguous rows; CTAs split each
+//   block into 16 KB slices so even a handful of pairs spreads over many SMs.
+#ifndef PAGEDATTN_CACHE_OPS_CUH
+#define PAGEDATTN_CACHE_OPS_CUH
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace pa {
+
+__global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                                     const int64_t* __restrict__ slots, uint4* k_cache,
+                                                     uint4* v_cache, int64_t num_slots, int row_vecs) {
+  const int t = blockIdx.x;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) set_device_error(DEVERR_BAD_SLOT);
+    return;
+  }
+  const uint4* src = (blockIdx.y ? v_new : k_new) + static_cast<int64_t>(t) * row_vecs;
+  uint4* dst = (blockIdx.y ? v_cache : k_cache) + slot * row_vecs;
+  for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) dst[i] = src[i];
+}
+
+constexpr int kCopySliceVecs = 1024;   // 16 KB per CTA slice
+
+__global__ void __launch_bounds__(256) copy_kernel(uint4* k_cache, uint4* v_cache, const int32_t* __restrict__ pairs,
+                                                   int num_blocks, int block_vecs) {
+  const int pi = blockIdx.x;
+  const int src = pairs[2 * pi];
+  const int dst = pairs[2 * pi + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) set_device_error(DEVERR_BAD_PAIR);
+    return;
+  }
+  uint4* cache = blockIdx.y ? v_cache : k_cache;
+  const uint4* s = cache + static_cast<int64_t>(src) * block_vecs;
+  uint4* d = cache + static_cast<int64_t>(dst) * block_vecs;
+  const int begin = blockIdx.z * kCopySliceVecs;
+  const int end = min(block_vecs, begin + kCopySliceVecs);
+  for (int i = begin + threadIdx.x; i < end; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace pa
+
+#endif

@@ -1,0 +1,350 @@
+// Device entry points of libpagedattn.so (declared in include/pa.h): argument
+// checks, launch configuration, TMA tensor maps, and the device error word.
+// All kernels live in this one translation unit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+
+#include "cache_ops.cuh"
+#include "decode.cuh"
+#include "pa.h"
+#include "pa_common.h"
+
+namespace {
+
+size_t elem_bytes(pa_dtype d) { return d == PA_F32 ? 4 : 2; }
+bool dtype_ok(int d) { return d == PA_F32 || d == PA_F16 || d == PA_BF16; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  return pa::fail(PA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+pa_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev].sms > 0) {
+    *out = cache[dev];
+    return PA_OK;
+  }
+  DeviceInfo d;
+  e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (dev < 64) cache[dev] = d;
+  *out = d;
+  return PA_OK;
+}
+
+// Optional tuning overrides (no effect on results): KV heads per CTA tile and
+// pipeline depth of the decode kernel.
+int env_int(const char* name) {
+  const char* v = std::getenv(name);
+  return v ? std::atoi(v) : 0;
+}
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  int num_blocks;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  int S, Hq, Hkv, D, BS;
+  float scale;
+  int P;
+  void* workspace;
+  void* out;
+  pa_dtype dtype;
+  cudaStream_t stream;
+};
+
+int max_parts(int max_blocks, int block_size, int P) {
+  if (P <= 0) return 1;
+  const long long cap = static_cast<long long>(max_blocks) * block_size;
+  return static_cast<int>((cap + P - 1) / P);
+}
+
+template <typename T>
+CUtensorMapDataType map_type();
+template <>
+CUtensorMapDataType map_type<float>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT32; }
+template <>
+CUtensorMapDataType map_type<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
+template <>
+CUtensorMapDataType map_type<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
+
+// Tensor map over one cache viewed as [num_blocks*block_size][Hkv][D], boxes of
+// 16 tokens x `tile_heads` heads x D.
+template <typename T>
+pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, long long rows, int tile_heads) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * sizeof(T),
+                                 static_cast<cuuint64_t>(Hkv) * D * sizeof(T)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(tile_heads),
+                             static_cast<cuuint32_t>(pa::kChunkTokens)};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+  return PA_OK;
+}
+
+template <typename T, int D, int G>
+pa_status launch_decode(const DecodeArgs& a) {
+  DeviceInfo dev;
+  pa_status st = device_info(&dev);
+  if (st != PA_OK) return st;
+
+  // KV heads per tile: the largest power of two <= 8 dividing Hkv whose K+V
+  // stage stays within 64 KB.
+  int ht = 8;
+  while (ht > 1 && (a.Hkv % ht != 0 || 2ull * pa::kChunkTokens * ht * D * sizeof(T) > 65536ull)) ht >>= 1;
+  const int forced_ht = env_int("PA_DECODE_TILE_HEADS");
+  if (forced_ht > 0 && forced_ht <= pa::kMaxTileHeads && a.Hkv % forced_ht == 0) ht = forced_ht;
+
+  const size_t tile_bytes = static_cast<size_t>(pa::kChunkTokens) * ht * D * sizeof(T);
+  const size_t q_bytes = static_cast<size_t>(ht) * G * D * sizeof(T);
+  const size_t per_stage = 2 * tile_bytes + sizeof(pa::StageMeta) + 2 * sizeof(uint64_t);
+  const size_t fixed = 2 * q_bytes + 4 * sizeof(uint64_t) + 16;
+  int stages = static_cast<int>((static_cast<size_t>(dev.smem_optin) - fixed) / per_stage);
+  if (stages > 8) stages = 8;
+  const int forced_st = env_int("PA_DECODE_STAGES");
+  if (forced_st >= 2 && forced_st < stages) stages = forced_st;
+  if (stages < 2) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: stage does not fit in shared memory");
+  const size_t smem = stages * per_stage + fixed;
+
+  auto kern = pa::decode_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+  const int threads = (ht + 1) * 32;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (per_sm < 1) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: kernel does not fit on an SM");
+
+  const int n_tiles = a.Hkv / ht;
+  const int np = max_parts(a.max_blocks, a.BS, a.P);
+  const long long units_bound = static_cast<long long>(a.S) * n_tiles * np;
+  const long long slots = static_cast<long long>(dev.sms) * per_sm;
+  const int grid = static_cast<int>(units_bound < slots ? units_bound : slots);
+
+  CUtensorMap tm_k, tm_v;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
+  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, ht);
+  if (st != PA_OK) return st;
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, ht);
+  if (st != PA_OK) return st;
+
+  pa::DecodeParams prm;
+  prm.q = a.q;
+  prm.block_tables = a.block_tables;
+  prm.context_lens = a.context_lens;
+  prm.out = a.out;
+  const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
+  prm.part_acc = a.P > 0 ? static_cast<float*>(a.workspace) : nullptr;
+  prm.part_ml = a.P > 0 ? reinterpret_cast<float2*>(static_cast<float*>(a.workspace) + acc_elems) : nullptr;
+  prm.num_seqs = a.S;
+  prm.num_q_heads = a.Hq;
+  prm.num_kv_heads = a.Hkv;
+  prm.max_blocks = a.max_blocks;
+  prm.block_size = a.BS;
+  prm.num_blocks = a.num_blocks;
+  prm.partition_size = a.P;
+  prm.max_parts = np;
+  prm.tile_heads = ht;
+  prm.num_tiles = n_tiles;
+  prm.stages = stages;
+  prm.tile_bytes = static_cast<uint32_t>(tile_bytes);
+  prm.q_bytes = static_cast<uint32_t>(q_bytes);
+  prm.qk_scale = a.scale * 1.4426950408889634f;
+
+  kern<<<grid, threads, smem, a.stream>>>(tm_k, tm_v, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_kernel launch");
+
+  if (a.P > 0) {
+    pa::ReduceParams rp;
+    rp.context_lens = a.context_lens;
+    rp.part_acc = prm.part_acc;
+    rp.part_ml = prm.part_ml;
+    rp.out = a.out;
+    rp.num_seqs = a.S;
+    rp.num_q_heads = a.Hq;
+    rp.partition_size = a.P;
+    rp.max_parts = np;
+    rp.cap = a.max_blocks * a.BS;
+    pa::reduce_kernel<T, D><<<a.S, 256, 0, a.stream>>>(rp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "reduce_kernel launch");
+  }
+  return pa::ok();
+}
+
+template <typename T, int D>
+pa_status dispatch_group(const DecodeArgs& a) {
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_decode<T, D, 1>(a);
+    case 2: return launch_decode<T, D, 2>(a);
+    case 4: return launch_decode<T, D, 4>(a);
+    case 8: return launch_decode<T, D, 8>(a);
+    default: return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: Hq/Hkv must be 1, 2, 4 or 8");
+  }
+}
+
+template <typename T>
+pa_status dispatch_dim(const DecodeArgs& a) {
+  switch (a.D) {
+    case 64: return dispatch_group<T, 64>(a);
+    case 128: return dispatch_group<T, 128>(a);
+    default: return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: head_dim must be 64 or 128");
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_append_kv(const void* k_new, const void* v_new, const int64_t* slot_mapping, int32_t num_tokens,
+                       void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                       int32_t head_dim, pa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return pa::fail(PA_ERR_INVALID, "pa_append_kv: bad dtype");
+  if (num_tokens < 0 || num_blocks < 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return pa::fail(PA_ERR_INVALID, "pa_append_kv: bad sizes");
+  const size_t row_bytes = static_cast<size_t>(num_kv_heads) * head_dim * elem_bytes(dtype);
+  if (row_bytes % 16 != 0) return pa::fail(PA_ERR_UNSUPPORTED, "pa_append_kv: row bytes must be a multiple of 16");
+  if (num_tokens == 0) return pa::ok();
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
+    return pa::fail(PA_ERR_INVALID, "pa_append_kv: null pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return pa::fail(PA_ERR_INVALID, "pa_append_kv: pointers must be 16-byte aligned");
+  const int row_vecs = static_cast<int>(row_bytes / 16);
+  const int threads = row_vecs >= 256 ? 256 : ((row_vecs + 31) / 32) * 32;
+  dim3 grid(num_tokens, 2);
+  pa::append_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), static_cast<int64_t>(num_blocks) * block_size, row_vecs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "append_kernel launch");
+  return pa::ok();
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t num_pairs, int32_t num_blocks,
+                         int32_t block_size, int32_t num_kv_heads, int32_t head_dim, pa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return pa::fail(PA_ERR_INVALID, "pa_copy_blocks: bad dtype");
+  if (num_pairs < 0 || num_blocks < 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return pa::fail(PA_ERR_INVALID, "pa_copy_blocks: bad sizes");
+  const size_t block_bytes = static_cast<size_t>(block_size) * num_kv_heads * head_dim * elem_bytes(dtype);
+  if (block_bytes % 16 != 0) return pa::fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: block bytes must be a multiple of 16");
+  if (num_pairs == 0) return pa::ok();
+  if (!k_cache || !v_cache || !pairs) return pa::fail(PA_ERR_INVALID, "pa_copy_blocks: null pointer");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return pa::fail(PA_ERR_INVALID, "pa_copy_blocks: pointers must be 16-byte aligned");
+  const int block_vecs = static_cast<int>(block_bytes / 16);
+  dim3 grid(num_pairs, 2, (block_vecs + pa::kCopySliceVecs - 1) / pa::kCopySliceVecs);
+  pa::copy_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_blocks, block_vecs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "copy_kernel launch");
+  return pa::ok();
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+                                int32_t block_size, int32_t partition_size) {
+  if (partition_size <= 0 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 ||
+      block_size <= 0)
+    return 0;
+  const size_t np = static_cast<size_t>(max_parts(max_blocks_per_seq, block_size, partition_size));
+  return static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
+}
+
+pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_cache, int32_t num_blocks,
+                              const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, float scale, int32_t partition_size, void* workspace,
+                              size_t workspace_bytes, void* out, pa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return pa::fail(PA_ERR_INVALID, "pa_decode_attention: bad dtype");
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: need Hq a positive multiple of Hkv");
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0 || block_size <= 0)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: bad pool sizes");
+  if (block_size % pa::kChunkTokens != 0)
+    return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: block_size must be a multiple of 16");
+  if (static_cast<long long>(num_blocks) * block_size >= (1ll << 31) ||
+      static_cast<long long>(max_blocks_per_seq) * block_size >= (1ll << 31))
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: pool or table too large for 32-bit token indices");
+  if (partition_size < 0 || (partition_size > 0 && partition_size % block_size != 0))
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: partition_size must be 0 or a multiple of block_size");
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: scale must be finite");
+  if (num_seqs == 0) return pa::ok();
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: null pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: q, caches and out must be 16-byte aligned");
+  if (partition_size > 0) {
+    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size,
+                                                 partition_size);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+      return pa::fail(PA_ERR_INVALID, "pa_decode_attention: workspace missing, too small (need " +
+                                          std::to_string(need) + " bytes) or misaligned");
+  }
+  DecodeArgs a{q,        k_cache,      v_cache,     num_blocks, block_tables, max_blocks_per_seq,
+               context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,  block_size,
+               scale,    partition_size, workspace, out,         dtype,        static_cast<cudaStream_t>(stream)};
+  switch (dtype) {
+    case PA_F32: return dispatch_dim<float>(a);
+    case PA_F16: return dispatch_dim<__half>(a);
+    case PA_BF16: return dispatch_dim<__nv_bfloat16>(a);
+  }
+  return pa::fail(PA_ERR_INVALID, "pa_decode_attention: bad dtype");
+}
+
+pa_status pa_device_error(int32_t* code_out, int32_t reset) {
+  if (!code_out) return pa::fail(PA_ERR_INVALID, "pa_device_error: code_out is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, pa::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (reset) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+  }
+  *code_out = v;
+  return pa::ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,249 @@
+"""Python binding of libpagedattn.so (C ABI in include/pa.h).
+
+Argument marshalling only: every step of the decode path runs in the
+library's CUDA kernels or its host pool.  Device arguments are torch CUDA
+tensors (their ``data_ptr()`` is passed); the stream is torch's current
+stream unless one is given.  Importing this module loads the library and
+raises ``ImportError`` when it has not been built -- there is no fallback.
+
+Function names match the C entry points.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        "libpagedattn.so is not built (expected at %s); run `python -m paged_kv_cache_341_b200.build`" % _LIB_PATH)
+_lib = ctypes.CDLL(_LIB_PATH)
+
+PA_OK, PA_ERR_EXHAUSTED, PA_ERR_INVALID, PA_ERR_REFCOUNT, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_UNSUPPORTED = range(7)
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+DTYPE_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+
+# Every symbol include/pa.h declares, with its C signature.
+_i32, _i64, _sz, _vp, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+_p32 = ctypes.POINTER(ctypes.c_int32)
+_p64 = ctypes.POINTER(ctypes.c_int64)
+SIGNATURES = {
+    "pa_pool_create": (_i32, [_i32, _i32, _p32, ctypes.POINTER(_vp)]),
+    "pa_pool_destroy": (None, [_vp]),
+    "pa_pool_alloc": (_i32, [_vp, _i32, _p32]),
+    "pa_pool_free": (_i32, [_vp, _p32, _i32]),
+    "pa_pool_fork": (_i32, [_vp, _p32, _i32]),
+    "pa_pool_refcount": (_i32, [_vp, _i32, _p32]),
+    "pa_pool_num_free": (_i32, [_vp, _p32]),
+    "pa_pool_export": (_i32, [_vp, _p32, _p32, _p32]),
+    "pa_seq_reserve_slot": (_i32, [_vp, _p32, _i32, _p32, _p64, _p32, _p32]),
+    "pa_reserve_slots": (_i32, [_vp, _p32, _i32, _p32, _i32, _p64, _p32, _p32]),
+    "pa_append_kv": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
+    "pa_decode_attention": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
+                                   _vp, _sz, _vp, _i32, _vp]),
+    "pa_device_error": (_i32, [_p32, _i32]),
+    "pa_last_error": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("status %d: %s" % (status, message))
+        self.status = status
+
+
+class PoolExhausted(PagedAttnError):
+    """No free block is left (the pages' "KV cache exhausted")."""
+
+
+def library_path():
+    return _LIB_PATH
+
+
+def pa_last_error():
+    return _lib.pa_last_error().decode()
+
+
+def _check(status):
+    if status != PA_OK:
+        cls = PoolExhausted if status == PA_ERR_EXHAUSTED else PagedAttnError
+        raise cls(status, pa_last_error())
+
+
+def _i32_array(values):
+    arr = np.ascontiguousarray(np.asarray(values, dtype=np.int32))
+    return arr, arr.ctypes.data_as(_p32)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev(t, name, dtype=None):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must have dtype %s, got %s" % (name, dtype, t.dtype))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# --------------------------------------------------------------------------
+# Host block pool
+# --------------------------------------------------------------------------
+
+class Pool:
+    """Refcounted block pool (pa_pool_*).  Host memory only; not thread-safe."""
+
+    def __init__(self, num_blocks, block_size, initial_free_order=None):
+        handle = ctypes.c_void_p()
+        if initial_free_order is None:
+            _check(_lib.pa_pool_create(num_blocks, block_size, None, ctypes.byref(handle)))
+        else:
+            arr, ptr = _i32_array(initial_free_order)
+            if arr.size != num_blocks:
+                raise ValueError("initial_free_order must have num_blocks entries")
+            _check(_lib.pa_pool_create(num_blocks, block_size, ptr, ctypes.byref(handle)))
+        self._h = handle
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            _lib.pa_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def pa_pool_alloc(self, n):
+        out = np.empty(max(n, 0), np.int32)
+        _check(_lib.pa_pool_alloc(self._h, n, out.ctypes.data_as(_p32)))
+        return out
+
+    def pa_pool_free(self, ids):
+        arr, ptr = _i32_array(ids)
+        _check(_lib.pa_pool_free(self._h, ptr, arr.size))
+
+    def pa_pool_fork(self, ids):
+        arr, ptr = _i32_array(ids)
+        _check(_lib.pa_pool_fork(self._h, ptr, arr.size))
+
+    def pa_pool_refcount(self, block_id):
+        out = ctypes.c_int32()
+        _check(_lib.pa_pool_refcount(self._h, block_id, ctypes.byref(out)))
+        return out.value
+
+    def pa_pool_num_free(self):
+        out = ctypes.c_int32()
+        _check(_lib.pa_pool_num_free(self._h, ctypes.byref(out)))
+        return out.value
+
+    def pa_pool_export(self):
+        refs = np.empty(self.num_blocks, np.int32)
+        free = np.empty(self.num_blocks, np.int32)
+        n = ctypes.c_int32()
+        _check(_lib.pa_pool_export(self._h, refs.ctypes.data_as(_p32), free.ctypes.data_as(_p32), ctypes.byref(n)))
+        return refs, free[: n.value].copy()
+
+    def pa_seq_reserve_slot(self, table, length):
+        """``table``: writable int32 numpy array (the sequence's row).  Returns (slot, new_len, src, dst)."""
+        if table.dtype != np.int32 or not table.flags.c_contiguous:
+            raise TypeError("table must be a contiguous int32 array")
+        n = ctypes.c_int32(length)
+        slot = ctypes.c_int64()
+        src, dst = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.pa_seq_reserve_slot(self._h, table.ctypes.data_as(_p32), table.size, ctypes.byref(n),
+                                        ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst)))
+        return slot.value, n.value, src.value, dst.value
+
+    def pa_reserve_slots(self, tables, lens):
+        """One step for every row of ``tables`` ([S, cap] int32, in place) and ``lens`` ([S] int32, in place).
+
+        Returns (slots int64 [S], pairs int32 [P, 2]).
+        """
+        if tables.dtype != np.int32 or lens.dtype != np.int32 or not tables.flags.c_contiguous:
+            raise TypeError("tables and lens must be contiguous int32 arrays")
+        s = lens.size
+        slots = np.empty(s, np.int64)
+        pairs = np.empty((max(s, 1), 2), np.int32)
+        npairs = ctypes.c_int32()
+        _check(_lib.pa_reserve_slots(self._h, tables.ctypes.data_as(_p32), tables.shape[1],
+                                     lens.ctypes.data_as(_p32), s, slots.ctypes.data_as(_p64),
+                                     pairs.ctypes.data_as(_p32), ctypes.byref(npairs)))
+        return slots, pairs[: npairs.value].copy()
+
+
+# --------------------------------------------------------------------------
+# Device kernels
+# --------------------------------------------------------------------------
+
+def pa_append_kv(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None):
+    """k_new/v_new [T, Hkv, D], slot_mapping int64 [T] (CUDA), caches [NB, bs, Hkv, D]."""
+    nb, bs, hkv, d = k_cache.shape
+    code = DTYPE_CODE[k_cache.dtype]
+    _check(_lib.pa_append_kv(_dev(k_new, "k_new", k_cache.dtype), _dev(v_new, "v_new", k_cache.dtype),
+                             _dev(slot_mapping, "slot_mapping", torch.int64), slot_mapping.numel(),
+                             _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype), nb, bs, hkv, d, code,
+                             _stream(stream)))
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
+    """pairs: int32 CUDA tensor [P, 2] of (src, dst) block ids."""
+    nb, bs, hkv, d = k_cache.shape
+    code = DTYPE_CODE[k_cache.dtype]
+    _check(_lib.pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
+                               _dev(pairs, "pairs", torch.int32), pairs.shape[0] if pairs.numel() else 0, nb, bs, hkv,
+                               d, code, _stream(stream)))
+
+
+def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size):
+    return int(_lib.pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size,
+                                             partition_size))
+
+
+def decode_workspace(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size, device=None):
+    """Allocate (through torch) the workspace pa_decode_attention needs; None when none is needed."""
+    nbytes = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size)
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale, out, partition_size=0,
+                        workspace=None, stream=None):
+    """q, out [S, Hq, D]; caches [NB, bs, Hkv, D]; block_tables int32 [S, MB]; context_lens int32 [S]."""
+    s, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != (s, hq, d):
+        raise ValueError("shape mismatch between q, caches and out")
+    code = DTYPE_CODE[k_cache.dtype]
+    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_decode_attention(_dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+                                    _dev(v_cache, "v_cache", k_cache.dtype), nb,
+                                    _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                                    _dev(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, float(scale),
+                                    int(partition_size), ws_ptr, ws_bytes, _dev(out, "out", k_cache.dtype), code,
+                                    _stream(stream)))
+
+
+def pa_device_error(reset=True):
+    """Synchronise and return the device error word (0 = no bad index seen)."""
+    code = ctypes.c_int32()
+    _check(_lib.pa_device_error(ctypes.byref(code), 1 if reset else 0))
+    return code.value

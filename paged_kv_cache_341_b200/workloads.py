@@ -49,7 +49,7 @@ class Workload:
     num_blocks: int = 0              # filled by lengths()
     max_blocks_per_seq: int = 0      # filled by lengths()
     shared_prefix: int = 0           # tokens shared by every sequence
-    append_headroom: int = 64        # tokens each sequence may still grow by
+    append_headroom: int = 128       # tokens each sequence may still grow by
 
     @property
     def seed(self):
