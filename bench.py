@@ -295,6 +295,7 @@ def run_ours(args):
     out = torch.empty((sc.batch, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device="cuda")
     ws = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
     kv_bytes = sc.kv_bytes()
+    config = workload_config(sc, args)
     launches_per_step = (1 if pairs.shape[0] else 0) + 1 + (2 if part > 0 else 1)
 
     def step(ev0=None, ev1=None):
@@ -402,7 +403,7 @@ def run_ours(args):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": workload_config(sc, args),
+            "config": config,
             "pct_of_hbm_peak": round(100 * value / world / peak, 2),
             "pct_of_8tbs_spec": round(100 * value / world / 8000.0, 2),
             "decode_tokens_per_s": round(world * sc.batch / (ms / 1e3), 1),

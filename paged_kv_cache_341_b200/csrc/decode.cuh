@@ -85,7 +85,9 @@ __device__ __forceinline__ int parts_of(int len, int psize) {
 }
 
 template <typename T, int D, int G>
-__global__ void __maxnreg__(224)
+// 8 consumer warps + 1 producer: three warps share one SM sub-partition, whose
+// 16K-register file caps a thread at 168 registers.
+__global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeParams prm) {
   constexpr int L = Lanes<D, G>::L;       // lanes per token
@@ -276,6 +278,13 @@ __global__ void __maxnreg__(224)
           mbar_arrive(&full[stage]);
         }
         __syncwarp();
+        // the marker is an arming of this stage too: the drain below walks
+        // back from the newest arming of every stage
+        ++armed;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
     }
     // Drain: every tile or query copy issued must have landed before exit.
