@@ -192,6 +192,40 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
                               int32_t partition_size, void* workspace, size_t workspace_bytes,
                               void* out, pa_dtype dtype, void* stream);
 
+/* Largest workspace pa_decode_attention_static can use: 32 MiB. */
+#define PA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
+
+/* pa_decode_attention for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this call; it exists for the library's users.
+ *
+ * Some callers cannot call cudaMalloc: a host framework that has already
+ * handed the whole GPU to its own allocator (so a fresh allocation would fail
+ * or fragment that pool), or code on a path where cudaMalloc's implicit
+ * device-wide synchronisation is not acceptable.  Such callers still own q,
+ * the caches, tables, lengths and out, but pass no workspace: the partials of
+ * the split-context path live in a static device array of
+ * PA_STATIC_WORKSPACE_BYTES that every GPU loading this library holds until
+ * the process exits.  This call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *
+ * Arguments and results are those of pa_decode_attention without
+ * `workspace`/`workspace_bytes`.  PA_ERR_INVALID, with a message naming the
+ * size, when pa_decode_workspace_size(...) for these sizes exceeds
+ * PA_STATIC_WORKSPACE_BYTES (partition_size == 0 needs none).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All calls
+ * on a device share the one array, which keeps whatever the last call left in
+ * it (nothing in it has to start at zero: every partial is written before it
+ * is read within a call).  Calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race on it; serialise them. */
+pa_status pa_decode_attention_static(const void* q, const void* k_cache, const void* v_cache,
+                                     int32_t num_blocks, const int32_t* block_tables,
+                                     int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                     int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                     int32_t head_dim, int32_t block_size, float scale,
+                                     int32_t partition_size, void* out, pa_dtype dtype, void* stream);
+
 /* Read (and, if reset != 0, clear) the device error word of the current
  * device: 0 = none; 1 = block id outside the pool in a table; 2 =
  * context length beyond the table; 3 = append slot outside the cache; 4 =

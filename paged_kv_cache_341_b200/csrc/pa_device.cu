@@ -331,6 +331,61 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
   return pa::fail(PA_ERR_INVALID, "pa_decode_attention: bad dtype");
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Workspace for pa_decode_attention_static: one fixed device array per GPU,
+// alive until the process exits, so that call never allocates.
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device (the host-side symbol is only a stand-in, not a device address).
+pa_status static_workspace(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention_static: device index >= 64");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_attention_static(const void* q, const void* k_cache, const void* v_cache, int32_t num_blocks,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size, float scale,
+                                     int32_t partition_size, void* out, pa_dtype dtype, void* stream) {
+  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size,
+                                               partition_size);
+  if (need > PA_STATIC_WORKSPACE_BYTES)
+    return pa::fail(PA_ERR_INVALID, "pa_decode_attention_static: these sizes need " + std::to_string(need) +
+                                        " bytes of workspace, more than the static " +
+                                        std::to_string(PA_STATIC_WORKSPACE_BYTES) +
+                                        "; use pa_decode_attention with a caller-allocated workspace");
+  void* ws = nullptr;
+  if (need > 0) {
+    pa_status st = static_workspace(&ws);
+    if (st != PA_OK) return st;
+  }
+  return pa_decode_attention(q, k_cache, v_cache, num_blocks, block_tables, max_blocks_per_seq, context_lens,
+                             num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale, partition_size, ws,
+                             need > 0 ? PA_STATIC_WORKSPACE_BYTES : 0, out, dtype, stream);
+}
+
 pa_status pa_device_error(int32_t* code_out, int32_t reset) {
   if (!code_out) return pa::fail(PA_ERR_INVALID, "pa_device_error: code_out is NULL");
   cudaError_t e = cudaDeviceSynchronize();

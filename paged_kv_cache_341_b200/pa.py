@@ -45,6 +45,8 @@ SIGNATURES = {
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "pa_decode_attention": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
                                    _vp, _sz, _vp, _i32, _vp]),
+    "pa_decode_attention_static": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32,
+                                          _i32, _vp, _i32, _vp]),
     "pa_device_error": (_i32, [_p32, _i32]),
     "pa_last_error": (ctypes.c_char_p, []),
 }
@@ -240,6 +242,32 @@ def pa_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale, 
                                     _dev(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, float(scale),
                                     int(partition_size), ws_ptr, ws_bytes, _dev(out, "out", k_cache.dtype), code,
                                     _stream(stream)))
+
+
+STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024
+
+
+def pa_decode_attention_static(q, k_cache, v_cache, block_tables, context_lens, scale, out, partition_size=0,
+                               stream=None):
+    """pa_decode_attention with no workspace argument, for callers that cannot allocate device memory.
+
+    The split-context partials go to a static 32 MiB device array inside the
+    library (shared by every call on the device; overlapping calls race), so
+    nothing is allocated here or in the library.  Sizes whose workspace would
+    exceed 32 MiB are rejected.  The first call on a device looks the array up
+    and should come before any stream capture.
+    """
+    s, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != (s, hq, d):
+        raise ValueError("shape mismatch between q, caches and out")
+    code = DTYPE_CODE[k_cache.dtype]
+    _check(_lib.pa_decode_attention_static(_dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+                                           _dev(v_cache, "v_cache", k_cache.dtype), nb,
+                                           _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                                           _dev(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs,
+                                           float(scale), int(partition_size), _dev(out, "out", k_cache.dtype), code,
+                                           _stream(stream)))
 
 
 def pa_device_error(reset=True):
