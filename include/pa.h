@@ -150,10 +150,11 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
                          int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
                          int32_t head_dim, pa_dtype dtype, void* stream);
 
-/* Bytes of device workspace pa_decode_attention needs for these sizes: 0 when
- * partition_size == 0, else room for one float32 partial (max, sum, D values)
- * per (sequence, query head, partition), partitions = ceil(max_blocks_per_seq
- * * block_size / partition_size). */
+/* Bytes of device workspace pa_decode_attention takes for these sizes: 256
+ * bytes for the work-unit counter, plus, when partition_size > 0, one float32
+ * partial (max, sum, D values) per (sequence, query head, partition), with
+ * partitions = ceil(max_blocks_per_seq * block_size / partition_size).  0 for
+ * invalid sizes. */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_blocks_per_seq, int32_t block_size,
                                 int32_t partition_size);
@@ -179,8 +180,14 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *   partition_size 0: one pass over each whole context.  > 0 (a multiple of
  *                  block_size): split each context into partitions of
  *                  that many tokens, compute partial (max, sum, output) per
- *                  partition and merge them with a second kernel; needs
- *                  `workspace` of pa_decode_workspace_size() bytes.
+ *                  partition and merge them with a second kernel.
+ *   workspace      device buffer of pa_decode_workspace_size() bytes, owned
+ *                  by the caller; required when partition_size > 0.  With a
+ *                  workspace the work units are handed out through a counter
+ *                  in it (zeroed by a 4-byte memset on `stream` before each
+ *                  launch); with NULL (only when partition_size == 0) they are
+ *                  dealt round-robin.  Calls sharing a workspace must not
+ *                  overlap on the GPU.
  * Supported: head_dim 64 or 128; Hq/Hkv in {1,2,4,8}; block_size a multiple
  * of 16; dtype f32/f16/bf16.  Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED,
  * PA_ERR_CUDA. */

@@ -10,28 +10,37 @@
 // Design (HBM-bound: every K/V byte is read exactly once):
 //
 // * Work unit = (sequence, partition of `partition_size` tokens, tile of HT
-//   KV heads).  Units are numbered sequence-major and dealt to a persistent
-//   grid (one or two CTAs per SM) in round-robin order, so neighbouring CTAs
-//   read neighbouring head tiles of the same blocks at about the same time.
-// * One producer warp streams each unit as chunks of 16 tokens.  A chunk is
-//   one TMA tile load per K and per V (box = 16 tokens x HT heads x D), taken
-//   straight from the physical block that the block table names; the table
-//   slice is held in the producer's registers, 32 entries per warp load.  The
-//   unit's HT*G query rows come in by one bulk copy into a double buffer.
-//   Stages are guarded by full/empty mbarriers.
-// * Consumer warp j handles KV head j of the tile for all G = Hq/Hkv query
-//   heads that share it, so each K/V element loaded serves G heads.  Lanes
-//   form groups of L lanes per token (L*E = D; each lane holds E elements of
-//   q for all G heads, as float32 pairs); a group's dot products finish with
-//   log2(L) xor-shuffles.  Every group keeps its own online-softmax state
-//   (reference max m, sum l, unnormalised output), merged across groups at the
-//   end of the unit, so the token loop has no cross-group traffic.
-// * The reference max is only moved when a score exceeds it by more than
-//   kTau = 8 (base-2 units): exp2(score - m) then stays <= 256, and the final
-//   division by l cancels the choice of m exactly, so rescaling of the
-//   accumulators is rare.
+//   KV heads).  Units are numbered in two passes over the sequences -- first
+//   every full partition, then every sequence's shorter remainder partition --
+//   and a persistent grid (one CTA per SM) takes them from an atomic counter
+//   in that order, so the small units come last and the SMs finish together.
+//   Without a workspace the units are dealt round-robin instead.
+// * One producer warp streams each unit as chunks of 16 tokens, each chunk
+//   taken straight from the physical block the block table names, by TMA tile
+//   loads into a ring of shared-memory stages guarded by full/empty mbarriers.
+//   The table slice sits in the producer's registers (32 entries per warp
+//   load); the unit's HT*G query rows come in by one bulk copy into a double
+//   buffer.
+// * Consumer warp j owns KV head j of the tile and all G = Hq/Hkv query heads
+//   that share it, so every K/V element loaded serves G query heads.  Two
+//   consumers exist:
+//   - decode_kernel (CUDA cores; float32 caches): lanes form groups of L
+//     lanes per token, each lane holding E = D/L elements of the G query rows
+//     as float32 pairs; dot products finish with log2(L) xor-shuffles, and
+//     each group keeps its own online-softmax state, merged at unit end.
+//   - decode_mma_kernel (tensor cores, mma.sync m16n8k16; 16-bit caches):
+//     S^T = K Q^T with the 16 tokens of a chunk as rows and the query heads
+//     as 8 columns, then O^T += V^T P^T with D as rows; K/V tiles arrive
+//     128-byte swizzled so ldmatrix reads them without bank conflicts, and P
+//     is transposed in registers with movmatrix.  Accumulation is float32; P
+//     is rounded to the cache's 16-bit type for the second product, and the
+//     softmax denominator sums the same rounded weights.
+// * Online softmax keeps a reference max m, moved only when a score exceeds
+//   it by more than kTau = 8 (base-2 units): exp2(score - m) stays <= 256 and
+//   the final division by l cancels the choice of m exactly, so accumulator
+//   rescaling is rare.
 // * With partitions, each unit writes its (m, l, unnormalised output) in
-//   float32 and a second kernel merges them; sequences that fit in one
+//   float32 and reduce_kernel merges them; sequences that fit in one
 //   partition are written out directly.
 #ifndef PAGEDATTN_DECODE_CUH
 #define PAGEDATTN_DECODE_CUH
@@ -47,6 +56,8 @@ namespace pa {
 constexpr int kChunkTokens = 16;      // tokens per pipeline stage
 constexpr float kTau = 8.0f;          // allowed growth of a score over the reference max (base 2)
 constexpr int kMaxTileHeads = 8;      // KV heads per CTA tile (consumer warps)
+constexpr int kSwizzleBytes = 128;    // TMA swizzle span of the tensor-core path
+constexpr int kSmemAlign = 1024;      // alignment of the stage ring (swizzle atom)
 
 struct DecodeParams {
   const void* q;                 // [S][Hq][D]
@@ -55,6 +66,7 @@ struct DecodeParams {
   void* out;                     // [S][Hq][D]
   float* part_acc;               // [S][Hq][NP][D]   (partitioned mode)
   float2* part_ml;               // [S][Hq][NP]      (m in base-2 units, l)
+  int* sched;                    // unit counter (zeroed before launch), or null: static order
   int num_seqs, num_q_heads, num_kv_heads;
   int max_blocks, block_size, num_blocks;
   int partition_size;            // 0 = whole context in one unit
@@ -72,6 +84,307 @@ struct StageMeta {
 };
 constexpr int kFirst = 1, kLast = 2;
 
+__device__ __forceinline__ int parts_of(int len, int psize) {
+  return (psize > 0 && len > 0) ? (len + psize - 1) / psize : 1;
+}
+
+// Bytes of dynamic shared memory the pipeline layout needs.
+__host__ __device__ constexpr size_t pipeline_smem_bytes(int stages, size_t tile_bytes, size_t q_bytes) {
+  return kSmemAlign + stages * (2 * tile_bytes + sizeof(StageMeta) + 2 * sizeof(uint64_t)) + 2 * q_bytes +
+         4 * sizeof(uint64_t) + 16;
+}
+
+// Shared-memory layout of both kernels: K ring, V ring, query double buffer,
+// stage metadata, barriers, abort flag.  The rings start 1 KB aligned.
+template <typename T, int D, int G>
+struct Pipeline {
+  T* s_k;
+  T* s_v;
+  T* s_q;
+  StageMeta* meta;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* q_full;
+  uint64_t* q_empty;
+  volatile int* abort_flag;
+  int stages, ht, tile_elems;
+
+  __device__ __forceinline__ Pipeline(unsigned char* raw, const DecodeParams& prm) {
+    const uintptr_t base =
+        (reinterpret_cast<uintptr_t>(raw) + kSmemAlign - 1) & ~static_cast<uintptr_t>(kSmemAlign - 1);
+    ht = prm.tile_heads;
+    stages = prm.stages;
+    tile_elems = kChunkTokens * ht * D;
+    s_k = reinterpret_cast<T*>(base);
+    s_v = s_k + stages * tile_elems;
+    s_q = s_v + stages * tile_elems;
+    meta = reinterpret_cast<StageMeta*>(s_q + 2 * ht * G * D);
+    full = reinterpret_cast<uint64_t*>(meta + stages);
+    empty = full + stages;
+    q_full = empty + stages;
+    q_empty = q_full + 2;
+    abort_flag = reinterpret_cast<volatile int*>(q_empty + 2);
+  }
+
+  __device__ __forceinline__ void init() {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], ht);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], ht);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+};
+
+// Producer warp: walks this CTA's units and fills the stage ring.
+// kSwizzled: one TMA box of 16 tokens x 128 bytes (128B-swizzled) per
+// (head, 128-byte column block of D) -- the layout the tensor-core consumer
+// reads; otherwise one box of 16 tokens x HT heads x D per K and per V tile.
+template <typename T, int D, int G, bool kSwizzled>
+__device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const DecodeParams& prm,
+                                             const CUtensorMap* tm_k, const CUtensorMap* tm_v, int lane) {
+  constexpr int kHalves = D * static_cast<int>(sizeof(T)) / kSwizzleBytes;
+  constexpr int kBoxElems = kSwizzleBytes / static_cast<int>(sizeof(T));
+  if (lane == 0) {
+    prefetch_tensormap(tm_k);
+    prefetch_tensormap(tm_v);
+  }
+  const uint64_t policy = policy_evict_first();
+  const int S = prm.num_seqs;
+  const int MB = prm.max_blocks;
+  const int BS = prm.block_size;
+  const int cap = MB * BS;
+  const int P = prm.partition_size;
+  const int n_tiles = prm.num_tiles;
+  const int HT = pl.ht;
+  const int stages = pl.stages;
+
+  // Units come in two passes over the sequences: pass 0 holds every full
+  // partition (the whole sequence when P == 0), pass 1 every remainder
+  // partition (and the single unit of an empty sequence).  A window of 32
+  // sequences is walked at a time: lane i holds sequence win_s0 + i.
+  int pass = 0;
+  int win_s0 = 0, win_base = 0;
+  int my_len = 0, my_units = 0, my_incl = 0, win_total = 0;
+  auto load_window = [&]() {
+    const int s = win_s0 + lane;
+    my_len = 0;
+    my_units = 0;
+    if (s < S) {
+      int len = prm.context_lens[s];
+      if (len > cap || len < 0) {
+        if (pass == 0) set_device_error(DEVERR_BAD_LENGTH);
+        len = len < 0 ? 0 : cap;
+      }
+      my_len = len;
+      int n;
+      if (P == 0) {
+        n = pass == 0 ? 1 : 0;
+      } else if (pass == 0) {
+        n = len / P;
+      } else {
+        n = (len % P != 0 || len == 0) ? 1 : 0;
+      }
+      my_units = n * n_tiles;
+    }
+    my_incl = my_units;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, my_incl, off);
+      if (lane >= off) my_incl += v;
+    }
+    win_total = __shfl_sync(0xffffffffu, my_incl, 31);
+  };
+  load_window();
+
+  int stage = 0;
+  uint32_t phase = 0;
+  int units_done = 0;
+  long long armed = 0;               // stages armed so far (for the drain at exit)
+  int q_issued = 0;                  // query copies issued so far
+  int tw_seq = -1, tw_base = -1, tw_val = 0;
+  bool ok = true;
+
+  // Next unit index: from the shared counter, claimed one unit ahead by lane
+  // 0 so the atomic's round trip overlaps the current unit; round-robin when
+  // there is no counter.
+  int claimed = 0;
+  if (prm.sched && lane == 0) claimed = atomicAdd(prm.sched, 1);
+  int rr = blockIdx.x;
+
+  while (ok) {
+    int u;
+    if (prm.sched) {
+      u = __shfl_sync(0xffffffffu, claimed, 0);
+    } else {
+      u = rr;
+      rr += gridDim.x;
+    }
+    bool exhausted = false;
+    while (u >= win_base + win_total) {
+      win_base += win_total;
+      win_s0 += 32;
+      if (win_s0 >= S) {
+        if (pass == 1) {
+          exhausted = true;
+          break;
+        }
+        pass = 1;
+        win_s0 = 0;
+      }
+      load_window();
+    }
+    if (exhausted) break;
+    if (prm.sched && lane == 0) claimed = atomicAdd(prm.sched, 1);
+    const unsigned hit = __ballot_sync(0xffffffffu, win_base + my_incl > u);
+    const int hl = __ffs(hit) - 1;
+    const int seq = win_s0 + hl;
+    const int len = __shfl_sync(0xffffffffu, my_len, hl);
+    const int excl = __shfl_sync(0xffffffffu, my_incl - my_units, hl);
+    const int r = u - (win_base + excl);
+    int part, tile;
+    if (pass == 0) {
+      part = r / n_tiles;
+      tile = r - part * n_tiles;
+    } else {
+      part = len / P;
+      tile = r;
+    }
+    const int nparts = parts_of(len, P);
+    const int tok_begin = P > 0 ? part * P : 0;
+    const int tok_end = P > 0 ? min(len, tok_begin + P) : len;
+    const int nchunks = max(1, (tok_end - tok_begin + kChunkTokens - 1) / kChunkTokens);
+    const int qslot = units_done & 1;
+
+    // Query rows of this unit: [HT*G][D] contiguous in q.
+    if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_empty[qslot], ((units_done >> 1) & 1) ^ 1, pl.abort_flag))) {
+      ok = false;
+      break;
+    }
+    ++q_issued;
+    if (lane == 0) {
+      const char* src = static_cast<const char*>(prm.q) +
+                        (static_cast<size_t>(seq) * prm.num_q_heads + static_cast<size_t>(tile) * HT * G) * D *
+                            sizeof(T);
+      mbar_arrive_expect_tx(&pl.q_full[qslot], prm.q_bytes);
+      bulk_load(pl.s_q + qslot * HT * G * D, src, prm.q_bytes, &pl.q_full[qslot]);
+    }
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int tok = tok_begin + c * kChunkTokens;
+      const int ntok = max(0, min(kChunkTokens, tok_end - tok));
+      int phys = 0, within = 0;
+      if (ntok > 0) {
+        const int blk = tok / BS;
+        within = tok - blk * BS;
+        const int wb = blk & ~31;
+        if (seq != tw_seq || wb != tw_base) {
+          tw_seq = seq;
+          tw_base = wb;
+          const int idx = wb + lane;
+          tw_val = idx < MB ? prm.block_tables[static_cast<size_t>(seq) * MB + idx] : 0;
+        }
+        phys = __shfl_sync(0xffffffffu, tw_val, blk - wb);
+        if (phys < 0 || phys >= prm.num_blocks) {
+          if (lane == 0) set_device_error(DEVERR_BAD_BLOCK_ID);
+          phys = 0;
+        }
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        StageMeta m;
+        m.seq = seq;
+        m.part = part;
+        m.tile = tile;
+        m.ntok = ntok;
+        m.flags = (c == 0 ? kFirst : 0) | (c == nchunks - 1 ? kLast : 0);
+        m.nparts = nparts;
+        m.qslot = qslot;
+        m.pad = 0;
+        pl.meta[stage] = m;
+        if (ntok > 0) {
+          mbar_arrive_expect_tx(&pl.full[stage], 2 * prm.tile_bytes);
+        } else {
+          mbar_arrive(&pl.full[stage]);
+        }
+      }
+      __syncwarp();
+      if (ntok > 0) {
+        const int row = phys * BS + within;
+        T* dk = pl.s_k + stage * pl.tile_elems;
+        T* dv = pl.s_v + stage * pl.tile_elems;
+        if constexpr (kSwizzled) {
+          // lanes split the 2 * HT * kHalves boxes of this stage
+          const int nbox = HT * kHalves;
+          for (int b = lane; b < 2 * nbox; b += 32) {
+            const int kv = b >= nbox ? 1 : 0;
+            const int hb = b - kv * nbox;                 // head-in-tile * kHalves + column block
+            T* dst = (kv ? dv : dk) + hb * kChunkTokens * kBoxElems;
+            tma_load_3d(dst, kv ? tm_v : tm_k, &pl.full[stage], 0, tile * HT * kHalves + hb, row, policy);
+          }
+        } else {
+          if (lane == 0) {
+            tma_load_3d(dk, tm_k, &pl.full[stage], 0, tile * HT, row, policy);
+            tma_load_3d(dv, tm_v, &pl.full[stage], 0, tile * HT, row, policy);
+          }
+        }
+      }
+      ++armed;
+      if (++stage == stages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    ++units_done;
+  }
+
+  if (ok) {
+    // End-of-work marker for the consumers.
+    if (__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag))) {
+      if (lane == 0) {
+        pl.meta[stage].seq = -1;
+        mbar_arrive(&pl.full[stage]);
+      }
+      __syncwarp();
+      // the marker is an arming of this stage too: the drain below walks
+      // back from the newest arming of every stage
+      ++armed;
+      if (++stage == stages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
+  // Drain: every tile or query copy issued must have landed before exit.
+  if (lane == 0) {
+    int st = stage, ph = phase;
+    const long long back = armed < stages ? armed : stages;
+    for (long long k = 0; k < back; ++k) {
+      if (--st < 0) {
+        st = stages - 1;
+        ph ^= 1;
+      }
+      mbar_wait_drain(&pl.full[st], ph);
+    }
+    for (int k = 1; k <= 2 && k <= q_issued; ++k) {
+      const int un = q_issued - k;
+      mbar_wait_drain(&pl.q_full[un & 1], (un >> 1) & 1);
+    }
+  }
+  __syncwarp();
+}
+
+// ===========================================================================
+// CUDA-core consumer
+// ===========================================================================
+
 // Lanes per token for a head size / group size: enough that the per-lane
 // q + accumulator registers (2*G*D/L floats) stay at or below 128.
 template <int D, int G>
@@ -79,10 +392,6 @@ struct Lanes {
   static constexpr int L = (D * G / 64 > 8) ? D * G / 64 : 8;
   static_assert(L <= 32 && (32 % L) == 0, "unsupported head_dim / group size");
 };
-
-__device__ __forceinline__ int parts_of(int len, int psize) {
-  return (psize > 0 && len > 0) ? (len + psize - 1) / psize : 1;
-}
 
 template <typename T, int D, int G>
 // 8 consumer warps + 1 producer: three warps share one SM sub-partition, whose
@@ -98,216 +407,18 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   static_assert(NCH >= 1 && E % EPC == 0, "lane slice must be whole 16-byte chunks");
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  const int HT = prm.tile_heads;
-  const int stages = prm.stages;
-  const int tile_elems = kChunkTokens * HT * D;
-  T* s_k = reinterpret_cast<T*>(smem);
-  T* s_v = s_k + stages * tile_elems;
-  T* s_q = s_v + stages * tile_elems;                       // 2 x [HT*G][D]
-  StageMeta* meta = reinterpret_cast<StageMeta*>(s_q + 2 * HT * G * D);
-  uint64_t* full = reinterpret_cast<uint64_t*>(meta + stages);
-  uint64_t* empty = full + stages;
-  uint64_t* q_full = empty + stages;
-  uint64_t* q_empty = q_full + 2;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(q_empty + 2);
-
+  Pipeline<T, D, G> pl(smem, prm);
+  const int HT = pl.ht;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < stages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], HT);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], HT);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
+  if (threadIdx.x == 0) pl.init();
   __syncthreads();
 
   if (warp == HT) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-    }
-    const uint64_t policy = policy_evict_first();
-    const int S = prm.num_seqs;
-    const int MB = prm.max_blocks;
-    const int BS = prm.block_size;
-    const int cap = MB * BS;
-    const int P = prm.partition_size;
-    const int n_tiles = prm.num_tiles;
-
-    // Window of 32 sequences: lane i holds sequence win_s0 + i.
-    int win_s0 = 0, win_base = 0;
-    int my_len = 0, my_units = 0, my_incl = 0, win_total = 0;
-    auto load_window = [&]() {
-      const int s = win_s0 + lane;
-      my_len = 0;
-      my_units = 0;
-      if (s < S) {
-        int len = prm.context_lens[s];
-        if (len > cap || len < 0) {
-          set_device_error(DEVERR_BAD_LENGTH);
-          len = len < 0 ? 0 : cap;
-        }
-        my_len = len;
-        my_units = parts_of(len, P) * n_tiles;
-      }
-      my_incl = my_units;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, my_incl, off);
-        if (lane >= off) my_incl += v;
-      }
-      win_total = __shfl_sync(0xffffffffu, my_incl, 31);
-    };
-    load_window();
-
-    int stage = 0;
-    uint32_t phase = 0;
-    int units_done = 0;
-    long long armed = 0;               // stages armed so far (for the drain at exit)
-    int q_issued = 0;                  // query copies issued so far
-    int tw_seq = -1, tw_base = -1, tw_val = 0;
-    bool ok = true;
-
-    for (int u = blockIdx.x; ok; u += gridDim.x) {
-      bool exhausted = false;
-      while (u >= win_base + win_total) {
-        win_base += win_total;
-        win_s0 += 32;
-        if (win_s0 >= S) {
-          exhausted = true;
-          break;
-        }
-        load_window();
-      }
-      if (exhausted) break;
-      const unsigned hit = __ballot_sync(0xffffffffu, win_base + my_incl > u);
-      const int hl = __ffs(hit) - 1;
-      const int seq = win_s0 + hl;
-      const int len = __shfl_sync(0xffffffffu, my_len, hl);
-      const int excl = __shfl_sync(0xffffffffu, my_incl - my_units, hl);
-      const int r = u - (win_base + excl);
-      const int part = r / n_tiles;
-      const int tile = r - part * n_tiles;
-      const int nparts = parts_of(len, P);
-      const int tok_begin = P > 0 ? part * P : 0;
-      const int tok_end = P > 0 ? min(len, tok_begin + P) : len;
-      const int nchunks = max(1, (tok_end - tok_begin + kChunkTokens - 1) / kChunkTokens);
-      const int qslot = units_done & 1;
-
-      // Query rows of this unit: [HT*G][D] contiguous in q.
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[qslot], ((units_done >> 1) & 1) ^ 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      ++q_issued;
-      if (lane == 0) {
-        const char* src = static_cast<const char*>(prm.q) +
-                          (static_cast<size_t>(seq) * prm.num_q_heads + static_cast<size_t>(tile) * HT * G) * D *
-                              sizeof(T);
-        mbar_arrive_expect_tx(&q_full[qslot], prm.q_bytes);
-        bulk_load(s_q + qslot * HT * G * D, src, prm.q_bytes, &q_full[qslot]);
-      }
-
-      for (int c = 0; c < nchunks; ++c) {
-        const int tok = tok_begin + c * kChunkTokens;
-        const int ntok = max(0, min(kChunkTokens, tok_end - tok));
-        int phys = 0, within = 0;
-        if (ntok > 0) {
-          const int blk = tok / BS;
-          within = tok - blk * BS;
-          const int wb = blk & ~31;
-          if (seq != tw_seq || wb != tw_base) {
-            tw_seq = seq;
-            tw_base = wb;
-            const int idx = wb + lane;
-            tw_val = idx < MB ? prm.block_tables[static_cast<size_t>(seq) * MB + idx] : 0;
-          }
-          phys = __shfl_sync(0xffffffffu, tw_val, blk - wb);
-          if (phys < 0 || phys >= prm.num_blocks) {
-            if (lane == 0) set_device_error(DEVERR_BAD_BLOCK_ID);
-            phys = 0;
-          }
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          StageMeta m;
-          m.seq = seq;
-          m.part = part;
-          m.tile = tile;
-          m.ntok = ntok;
-          m.flags = (c == 0 ? kFirst : 0) | (c == nchunks - 1 ? kLast : 0);
-          m.nparts = nparts;
-          m.qslot = qslot;
-          m.pad = 0;
-          meta[stage] = m;
-          if (ntok > 0) {
-            mbar_arrive_expect_tx(&full[stage], 2 * prm.tile_bytes);
-            const int row = phys * BS + within;
-            tma_load_3d(s_k + stage * tile_elems, &tm_k, &full[stage], 0, tile * HT, row, policy);
-            tma_load_3d(s_v + stage * tile_elems, &tm_v, &full[stage], 0, tile * HT, row, policy);
-          } else {
-            mbar_arrive(&full[stage]);
-          }
-        }
-        __syncwarp();
-        ++armed;
-        if (++stage == stages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      ++units_done;
-    }
-
-    if (ok) {
-      // End-of-work marker for the consumers.
-      if (__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1, abort_flag))) {
-        if (lane == 0) {
-          meta[stage].seq = -1;
-          mbar_arrive(&full[stage]);
-        }
-        __syncwarp();
-        // the marker is an arming of this stage too: the drain below walks
-        // back from the newest arming of every stage
-        ++armed;
-        if (++stage == stages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-    // Drain: every tile or query copy issued must have landed before exit.
-    if (lane == 0) {
-      int st = stage, ph = phase;
-      const long long back = armed < stages ? armed : stages;
-      for (long long k = 0; k < back; ++k) {
-        if (--st < 0) {
-          st = stages - 1;
-          ph ^= 1;
-        }
-        mbar_wait_drain(&full[st], ph);
-      }
-      for (int k = 1; k <= 2 && k <= q_issued; ++k) {
-        const int un = q_issued - k;
-        mbar_wait_drain(&q_full[un & 1], (un >> 1) & 1);
-      }
-    }
-    __syncwarp();
+    run_producer<T, D, G, false>(pl, prm, &tm_k, &tm_v, lane);
     return;
   }
 
-  // -------------------------------------------------------------- consumers
   const int j = warp;                 // KV head within the tile
   const int grp = lane / L;           // token group
   const int li = lane % L;            // lane within the group
@@ -321,13 +432,13 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   int units_done = 0;
 
   while (true) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) return;
-    const StageMeta mt = meta[stage];
+    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag))) return;
+    const StageMeta mt = pl.meta[stage];
     if (mt.seq < 0) return;
 
     if (mt.flags & kFirst) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[mt.qslot], (units_done >> 1) & 1, abort_flag))) return;
-      const T* qrow = s_q + mt.qslot * HT * G * D + j * G * D;
+      if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag))) return;
+      const T* qrow = pl.s_q + mt.qslot * HT * G * D + j * G * D;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -342,12 +453,12 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
         for (int e = 0; e < E / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&q_empty[mt.qslot]);
+      if (lane == 0) mbar_arrive(&pl.q_empty[mt.qslot]);
     }
 
     if (mt.ntok > 0) {
-      const T* kt = s_k + stage * tile_elems + j * D;
-      const T* vt = s_v + stage * tile_elems + j * D;
+      const T* kt = pl.s_k + stage * pl.tile_elems + j * D;
+      const T* vt = pl.s_v + stage * pl.tile_elems + j * D;
       const int npass = (mt.ntok + NG - 1) / NG;
 #pragma unroll 1
       for (int pass = 0; pass < npass; ++pass) {
@@ -394,8 +505,8 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
-    if (++stage == stages) {
+    if (lane == 0) mbar_arrive(&pl.empty[stage]);
+    if (++stage == pl.stages) {
       stage = 0;
       phase ^= 1;
     }
@@ -464,9 +575,290 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   }
 }
 
+// ===========================================================================
+// Tensor-core consumer (16-bit caches)
+// ===========================================================================
+
+template <typename T>
+struct MmaType;
+template <>
+struct MmaType<__nv_bfloat16> {
+  __device__ __forceinline__ static void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  // (lo, hi) -> packed pair, rounded to nearest even
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+  }
+  __device__ __forceinline__ static float2 unpack(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+};
+template <>
+struct MmaType<__half> {
+  __device__ __forceinline__ static void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+  }
+  __device__ __forceinline__ static float2 unpack(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Transpose of an 8x8 16-bit matrix held one row pair per thread.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Byte offset, inside one 16-token x 128-byte swizzled box, of 16-byte chunk
+// `chunk` of token row `tok` (128B swizzle: chunk ^= row mod 8).
+__device__ __forceinline__ uint32_t swz(int tok, int chunk) {
+  return static_cast<uint32_t>(tok * kSwizzleBytes + ((chunk ^ (tok & 7)) << 4));
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const DecodeParams prm) {
+  static_assert(sizeof(T) == 2, "tensor-core consumer takes 16-bit caches");
+  static_assert(G >= 1 && G <= 8, "query heads per KV head must fit the 8 MMA columns");
+  constexpr int kHalves = D * 2 / kSwizzleBytes;            // 64-element column blocks
+  constexpr int kBoxBytes = kChunkTokens * kSwizzleBytes;   // one swizzled box (2 KB)
+  constexpr int KSTEPS = D / 16;                            // k-steps of S^T = K Q^T
+  constexpr int MTILES = D / 16;                            // m-tiles of O^T = V^T P^T
+  using M = MmaType<T>;
+
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Pipeline<T, D, G> pl(smem, prm);
+  const int HT = pl.ht;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) pl.init();
+  __syncthreads();
+
+  if (warp == HT) {
+    run_producer<T, D, G, true>(pl, prm, &tm_k, &tm_v, lane);
+    return;
+  }
+
+  const int j = warp;              // KV head within the tile
+  const int gq = lane >> 2;        // fragment row group
+  const int tq = lane & 3;         // fragment column pair
+  const int h0 = 2 * tq;           // this thread's two query-head columns h0, h0 + 1
+
+  // ldmatrix row addresses.  QK (A = K, rows = tokens): matrix i = lane/8
+  // covers tokens 8*(i%2).., column chunk i/2.  PV (A = V^T through .trans):
+  // matrix i covers tokens 8*(i/2).., column chunk i%2.
+  const int qk_tok = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int qk_chk = lane >> 4;
+  const int pv_tok = (lane & 7) + (lane >> 4) * 8;
+  const int pv_chk = (lane >> 3) & 1;
+
+  uint32_t qf[KSTEPS][2];          // B fragments of Q^T (query heads as the 8 columns)
+  float o[MTILES][4];              // O^T accumulators: rows D, columns heads
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  const uint32_t s_k0 = smem_addr(pl.s_k) + j * kHalves * kBoxBytes;
+  const uint32_t s_v0 = smem_addr(pl.s_v) + j * kHalves * kBoxBytes;
+  const uint32_t tile_bytes = prm.tile_bytes;
+
+  int stage = 0;
+  uint32_t phase = 0;
+  int units_done = 0;
+
+  while (true) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag))) return;
+    const StageMeta mt = pl.meta[stage];
+    if (mt.seq < 0) return;
+
+    if (mt.flags & kFirst) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag))) return;
+      const T* qbase = pl.s_q + mt.qslot * HT * G * D + j * G * D;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        if (gq < G) {
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(qbase + gq * D + kk * 16);
+          qf[kk][0] = row[tq];
+          qf[kk][1] = row[tq + 4];
+        } else {
+          qf[kk][0] = 0u;
+          qf[kk][1] = 0u;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pl.q_empty[mt.qslot]);
+#pragma unroll
+      for (int i = 0; i < MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+
+    if (mt.ntok > 0) {
+      const uint32_t kb = s_k0 + stage * tile_bytes;
+      const uint32_t vb = s_v0 + stage * tile_bytes;
+      // S^T[16 tokens][8 heads] = K Q^T
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        const int blk = (kk * 16) / 64;
+        const int chunk = ((kk * 16) % 64) / 8 + qk_chk;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kb + blk * kBoxBytes + swz(qk_tok, chunk), a0, a1, a2, a3);
+        M::mma(s, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+      }
+      // scores in base-2 units; tokens gq, gq+8 beyond the chunk are masked
+      const bool v_lo = gq < mt.ntok;
+      const bool v_hi = gq + 8 < mt.ntok;
+      const float x0 = v_lo ? s[0] * prm.qk_scale : -INFINITY;
+      const float x1 = v_lo ? s[1] * prm.qk_scale : -INFINITY;
+      const float x2 = v_hi ? s[2] * prm.qk_scale : -INFINITY;
+      const float x3 = v_hi ? s[3] * prm.qk_scale : -INFINITY;
+      const bool over = (x0 > m0 + kTau) | (x2 > m0 + kTau) | (x1 > m1 + kTau) | (x3 > m1 + kTau);
+      if (__any_sync(0xffffffffu, over)) {
+        // column maxima over the chunk's 16 tokens (the 8 lanes sharing tq)
+        float c0 = fmaxf(x0, x2), c1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          c0 = fmaxf(c0, __shfl_xor_sync(0xffffffffu, c0, off));
+          c1 = fmaxf(c1, __shfl_xor_sync(0xffffffffu, c1, off));
+        }
+        const float n0 = c0 > m0 + kTau ? c0 : m0;
+        const float n1 = c1 > m1 + kTau ? c1 : m1;
+        const float f0 = exp2_approx(m0 - n0);
+        const float f1 = exp2_approx(m1 - n1);
+        l0 *= f0;
+        l1 *= f1;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+          o[i][0] *= f0;
+          o[i][1] *= f1;
+          o[i][2] *= f0;
+          o[i][3] *= f1;
+        }
+        m0 = n0;
+        m1 = n1;
+      }
+      // P^T rounded to the 16-bit type; the denominator sums the same rounded values
+      const uint32_t p_lo = M::pack(exp2_approx(x0 - m0), exp2_approx(x1 - m1));   // token gq
+      const uint32_t p_hi = M::pack(exp2_approx(x2 - m0), exp2_approx(x3 - m1));   // token gq + 8
+      const float2 r_lo = M::unpack(p_lo), r_hi = M::unpack(p_hi);
+      l0 += r_lo.x + r_hi.x;
+      l1 += r_lo.y + r_hi.y;
+      const uint32_t b0 = movmatrix_trans(p_lo);     // P^T tokens 0-7 as B (k = tokens, n = heads)
+      const uint32_t b1 = movmatrix_trans(p_hi);     // P^T tokens 8-15
+      // rows of V beyond the chunk may hold anything: zero them in the fragments
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (mt.ntok < kChunkTokens) {
+        mlo = (2 * tq < mt.ntok ? 0x0000ffffu : 0u) | (2 * tq + 1 < mt.ntok ? 0xffff0000u : 0u);
+        mhi = (2 * tq + 8 < mt.ntok ? 0x0000ffffu : 0u) | (2 * tq + 9 < mt.ntok ? 0xffff0000u : 0u);
+      }
+      // O^T[D][heads] += V^T P^T
+#pragma unroll
+      for (int i = 0; i < MTILES; ++i) {
+        const int blk = (i * 16) / 64;
+        const int chunk = ((i * 16) % 64) / 8 + pv_chk;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(vb + blk * kBoxBytes + swz(pv_tok, chunk), a0, a1, a2, a3);
+        M::mma(o[i], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pl.empty[stage]);
+    if (++stage == pl.stages) {
+      stage = 0;
+      phase ^= 1;
+    }
+
+    if (mt.flags & kLast) {
+      // full column sums of l over the 8 row groups
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      const int hq0 = (mt.tile * HT + j) * G;
+      const bool w0 = h0 < G, w1 = h0 + 1 < G;
+      if (mt.nparts == 1) {
+        const float i0 = l0 > 0.f ? 1.0f / l0 : 0.f;
+        const float i1 = l1 > 0.f ? 1.0f / l1 : 0.f;
+        T* r0 = static_cast<T*>(prm.out) + (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq0 + h0) * D;
+        T* r1 = r0 + D;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+          const int d = i * 16 + gq;
+          if (w0) {
+            r0[d] = static_cast<T>(o[i][0] * i0);
+            r0[d + 8] = static_cast<T>(o[i][2] * i0);
+          }
+          if (w1) {
+            r1[d] = static_cast<T>(o[i][1] * i1);
+            r1[d + 8] = static_cast<T>(o[i][3] * i1);
+          }
+        }
+      } else {
+        const size_t p0 = (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq0 + h0) * prm.max_parts + mt.part;
+        const size_t p1 = p0 + prm.max_parts;
+        float* r0 = prm.part_acc + p0 * D;
+        float* r1 = prm.part_acc + p1 * D;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+          const int d = i * 16 + gq;
+          if (w0) {
+            r0[d] = o[i][0];
+            r0[d + 8] = o[i][2];
+          }
+          if (w1) {
+            r1[d] = o[i][1];
+            r1[d + 8] = o[i][3];
+          }
+        }
+        if (gq == 0) {
+          if (w0) prm.part_ml[p0] = make_float2(m0, l0);
+          if (w1) prm.part_ml[p1] = make_float2(m1, l1);
+        }
+      }
+      ++units_done;
+    }
+  }
+}
+
+// ===========================================================================
 // Merge of per-partition partials: M = max m_p, w_p = 2^(m_p - M),
-// out = sum_p w_p acc_p / sum_p w_p l_p.  One CTA per sequence; sequences
-// that fit one partition were written by decode_kernel and are skipped.
+// out = sum_p w_p acc_p / sum_p w_p l_p.  One warp per (sequence, query
+// head); sequences that fit one partition were written by the decode kernel
+// and are skipped.
+// ===========================================================================
 struct ReduceParams {
   const int32_t* context_lens;
   const float* part_acc;
@@ -475,49 +867,56 @@ struct ReduceParams {
   int num_seqs, num_q_heads, partition_size, max_parts, cap;
 };
 
+constexpr int kReduceWarps = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) reduce_kernel(const ReduceParams prm) {
+__global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceParams prm) {
   constexpr int PER = D / 32;                // contiguous elements per lane
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
-  const int s = blockIdx.x;
+  const int s = blockIdx.y;
   int len = prm.context_lens[s];
   len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
   const int np = parts_of(len, prm.partition_size);
   if (np <= 1) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int hq = warp; hq < prm.num_q_heads; hq += nwarps) {
-    const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + hq) * prm.max_parts;
-    float mx = -INFINITY;
-    for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hq = blockIdx.x * kReduceWarps + warp;
+  if (hq >= prm.num_q_heads) return;
+  const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + hq) * prm.max_parts;
+  float mx = -INFINITY;
+  for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float lsum = 0.f;
-    for (int p = lane; p < np; p += 32) {
-      const float2 ml = prm.part_ml[base + p];
-      lsum += ml.y * exp2_approx(ml.x - mx);
-    }
+  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float lsum = 0.f;
+  for (int p = lane; p < np; p += 32) {
+    const float2 ml = prm.part_ml[base + p];
+    lsum += ml.y * exp2_approx(ml.x - mx);
+  }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    float2 o[PER / 2];
+  for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  float2 o[PER / 2];
 #pragma unroll
-    for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
-    for (int p = 0; p < np; ++p) {
-      const float w = exp2_approx(prm.part_ml[base + p].x - mx);
-      const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p) * D + lane * PER);
+  for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
+  for (int p0 = 0; p0 < np; p0 += 32) {
+    const int pl = p0 + lane;
+    const float wl = pl < np ? exp2_approx(prm.part_ml[base + pl].x - mx) : 0.f;
+    const int n = min(32, np - p0);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + k) * D + lane * PER);
 #pragma unroll
       for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(w, w), src[e]);
     }
-    const float inv = 1.0f / lsum;
-    T* dst = static_cast<T*>(prm.out) + (static_cast<size_t>(s) * prm.num_q_heads + hq) * D + lane * PER;
+  }
+  const float inv = 1.0f / lsum;
+  T* dst = static_cast<T*>(prm.out) + (static_cast<size_t>(s) * prm.num_q_heads + hq) * D + lane * PER;
 #pragma unroll
-    for (int e = 0; e < PER / 2; ++e) {
-      fmul2(o[e], make_float2(inv, inv));
-      if constexpr (sizeof(T) == 4) {
-        reinterpret_cast<float2*>(dst)[e] = o[e];
-      } else if constexpr (Chunk<T>::kElems == 8 && sizeof(T) == 2) {
-        const uint32_t w = Chunk<T>::narrow(o[e]);
-        reinterpret_cast<uint32_t*>(dst)[e] = w;
-      }
+  for (int e = 0; e < PER / 2; ++e) {
+    fmul2(o[e], make_float2(inv, inv));
+    if constexpr (sizeof(T) == 4) {
+      reinterpret_cast<float2*>(dst)[e] = o[e];
+    } else {
+      reinterpret_cast<uint32_t*>(dst)[e] = Chunk<T>::narrow(o[e]);
     }
   }
 }

@@ -87,6 +87,8 @@ struct DecodeArgs {
   cudaStream_t stream;
 };
 
+constexpr size_t kSchedBytes = 256;   // unit counter at the head of the workspace
+
 int max_parts(int max_blocks, int block_size, int P) {
   if (P <= 0) return 1;
   const long long cap = static_cast<long long>(max_blocks) * block_size;
@@ -102,23 +104,46 @@ CUtensorMapDataType map_type<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 template <>
 CUtensorMapDataType map_type<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
 
-// Tensor map over one cache viewed as [num_blocks*block_size][Hkv][D], boxes of
-// 16 tokens x `tile_heads` heads x D.
+// Tensor map over one cache viewed as [num_blocks*block_size][Hkv][D].
+// Plain: boxes of 16 tokens x `tile_heads` heads x D.  Swizzled (tensor-core
+// consumer): the row viewed as Hkv*D/64 column blocks of 128 bytes, boxes of
+// 16 tokens x one column block, stored 128B-swizzled in shared memory.
 template <typename T>
-pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, long long rows, int tile_heads) {
+pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, long long rows, int tile_heads,
+                         bool swizzled) {
   auto encode = tensor_map_encoder();
   if (!encode) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * sizeof(T),
-                                 static_cast<cuuint64_t>(Hkv) * D * sizeof(T)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(tile_heads),
-                             static_cast<cuuint32_t>(pa::kChunkTokens)};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(Hkv) * D * sizeof(T);
   const cuuint32_t elem_strides[3] = {1, 1, 1};
-  CUresult r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r;
+  if (swizzled) {
+    const cuuint64_t box_elems = pa::kSwizzleBytes / sizeof(T);
+    const cuuint64_t dims[3] = {box_elems, static_cast<cuuint64_t>(Hkv) * D / box_elems,
+                                static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pa::kSwizzleBytes), row_bytes};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_elems), 1, static_cast<cuuint32_t>(pa::kChunkTokens)};
+    r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                                static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * sizeof(T), row_bytes};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(tile_heads),
+                               static_cast<cuuint32_t>(pa::kChunkTokens)};
+    r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (r != CUDA_SUCCESS) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
   return PA_OK;
+}
+
+// Consumer used for 16-bit caches: tensor cores unless PA_DECODE_PATH=alu
+// (the CUDA-core consumer, kept for float32 caches and for comparisons).
+bool use_tensor_cores() {
+  const char* v = std::getenv("PA_DECODE_PATH");
+  return !(v && std::string(v) == "alu");
 }
 
 template <typename T, int D, int G>
@@ -127,25 +152,32 @@ pa_status launch_decode(const DecodeArgs& a) {
   pa_status st = device_info(&dev);
   if (st != PA_OK) return st;
 
-  // KV heads per tile: the largest power of two <= 8 dividing Hkv whose K+V
-  // stage stays within 64 KB.
-  int ht = 8;
-  while (ht > 1 && (a.Hkv % ht != 0 || 2ull * pa::kChunkTokens * ht * D * sizeof(T) > 65536ull)) ht >>= 1;
+  // Launch shape, chosen by measurement on B200 (sweep over 1/2/4/8 KV heads
+  // per CTA x 2..6 stages on the four large workloads): one KV head per CTA
+  // and a 3-deep ring, i.e. small CTAs, about seven per SM, whose independent
+  // producers keep HBM busy, beat fewer, wider CTAs by up to 25%.
+  int ht = 1;
+  int stages = 3;
   const int forced_ht = env_int("PA_DECODE_TILE_HEADS");
   if (forced_ht > 0 && forced_ht <= pa::kMaxTileHeads && a.Hkv % forced_ht == 0) ht = forced_ht;
+  const int forced_st = env_int("PA_DECODE_STAGES");
+  if (forced_st >= 2 && forced_st <= 8) stages = forced_st;
 
   const size_t tile_bytes = static_cast<size_t>(pa::kChunkTokens) * ht * D * sizeof(T);
   const size_t q_bytes = static_cast<size_t>(ht) * G * D * sizeof(T);
-  const size_t per_stage = 2 * tile_bytes + sizeof(pa::StageMeta) + 2 * sizeof(uint64_t);
-  const size_t fixed = 2 * q_bytes + 4 * sizeof(uint64_t) + 16;
-  int stages = static_cast<int>((static_cast<size_t>(dev.smem_optin) - fixed) / per_stage);
-  if (stages > 8) stages = 8;
-  const int forced_st = env_int("PA_DECODE_STAGES");
-  if (forced_st >= 2 && forced_st < stages) stages = forced_st;
+  while (stages >= 2 && pa::pipeline_smem_bytes(stages, tile_bytes, q_bytes) > static_cast<size_t>(dev.smem_optin))
+    --stages;
   if (stages < 2) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: stage does not fit in shared memory");
-  const size_t smem = stages * per_stage + fixed;
+  const size_t smem = pa::pipeline_smem_bytes(stages, tile_bytes, q_bytes);
 
-  auto kern = pa::decode_kernel<T, D, G>;
+  bool mma = false;
+  void (*kern)(const CUtensorMap, const CUtensorMap, const pa::DecodeParams) = pa::decode_kernel<T, D, G>;
+  if constexpr (sizeof(T) == 2) {
+    if (use_tensor_cores()) {
+      kern = pa::decode_mma_kernel<T, D, G>;
+      mma = true;
+    }
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   const int threads = (ht + 1) * 32;
@@ -162,9 +194,9 @@ pa_status launch_decode(const DecodeArgs& a) {
 
   CUtensorMap tm_k, tm_v;
   const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
-  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, ht);
+  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, ht, mma);
   if (st != PA_OK) return st;
-  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, ht);
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, ht, mma);
   if (st != PA_OK) return st;
 
   pa::DecodeParams prm;
@@ -172,9 +204,12 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.block_tables = a.block_tables;
   prm.context_lens = a.context_lens;
   prm.out = a.out;
+  // workspace: [unit counter, 256 B][partial outputs][partial (m, l)]
   const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
-  prm.part_acc = a.P > 0 ? static_cast<float*>(a.workspace) : nullptr;
-  prm.part_ml = a.P > 0 ? reinterpret_cast<float2*>(static_cast<float*>(a.workspace) + acc_elems) : nullptr;
+  char* ws = static_cast<char*>(a.workspace);
+  prm.sched = ws ? reinterpret_cast<int*>(ws) : nullptr;
+  prm.part_acc = a.P > 0 ? reinterpret_cast<float*>(ws + kSchedBytes) : nullptr;
+  prm.part_ml = a.P > 0 ? reinterpret_cast<float2*>(prm.part_acc + acc_elems) : nullptr;
   prm.num_seqs = a.S;
   prm.num_q_heads = a.Hq;
   prm.num_kv_heads = a.Hkv;
@@ -190,6 +225,10 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.q_bytes = static_cast<uint32_t>(q_bytes);
   prm.qk_scale = a.scale * 1.4426950408889634f;
 
+  if (prm.sched) {
+    e = cudaMemsetAsync(prm.sched, 0, sizeof(int), a.stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(unit counter)");
+  }
   kern<<<grid, threads, smem, a.stream>>>(tm_k, tm_v, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_kernel launch");
@@ -205,7 +244,8 @@ pa_status launch_decode(const DecodeArgs& a) {
     rp.partition_size = a.P;
     rp.max_parts = np;
     rp.cap = a.max_blocks * a.BS;
-    pa::reduce_kernel<T, D><<<a.S, 256, 0, a.stream>>>(rp);
+    const dim3 rgrid((a.Hq + pa::kReduceWarps - 1) / pa::kReduceWarps, a.S);
+    pa::reduce_kernel<T, D><<<rgrid, pa::kReduceWarps * 32, 0, a.stream>>>(rp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "reduce_kernel launch");
   }
@@ -282,11 +322,12 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
 
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
                                 int32_t block_size, int32_t partition_size) {
-  if (partition_size <= 0 || num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 ||
-      block_size <= 0)
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||
+      partition_size < 0)
     return 0;
+  if (partition_size == 0) return kSchedBytes;
   const size_t np = static_cast<size_t>(max_parts(max_blocks_per_seq, block_size, partition_size));
-  return static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
+  return kSchedBytes + static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
 }
 
 pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_cache, int32_t num_blocks,
@@ -313,7 +354,7 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: null pointer");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: q, caches and out must be 16-byte aligned");
-  if (partition_size > 0) {
+  if (partition_size > 0 || workspace) {
     const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size,
                                                  partition_size);
     if (!workspace || workspace_bytes < need || !aligned16(workspace))
@@ -383,7 +424,7 @@ pa_status pa_decode_attention_static(const void* q, const void* k_cache, const v
   }
   return pa_decode_attention(q, k_cache, v_cache, num_blocks, block_tables, max_blocks_per_seq, context_lens,
                              num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale, partition_size, ws,
-                             need > 0 ? PA_STATIC_WORKSPACE_BYTES : 0, out, dtype, stream);
+                             ws ? PA_STATIC_WORKSPACE_BYTES : 0, out, dtype, stream);
 }
 
 pa_status pa_device_error(int32_t* code_out, int32_t reset) {

@@ -66,9 +66,10 @@ def test_decode_rejects_bad_arguments_on_host(built_library):
 
 def test_workspace_size_formula(built_library):
     from paged_kv_cache_341_b200 import pa
-    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 0) == 0
+    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 0) == 256
     np_ = -(-1026 * 32 // 512)
-    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 512) == 8 * 64 * np_ * (128 * 4 + 8)
+    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 512) == 256 + 8 * 64 * np_ * (128 * 4 + 8)
+    assert pa.pa_decode_workspace_size(0, 64, 128, 1026, 32, 512) == 0
 
 
 def test_cache_ops_reject_bad_arguments_on_host(built_library):

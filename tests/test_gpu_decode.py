@@ -28,7 +28,7 @@ def pa():
     return mod
 
 
-def run_decode(pa, dtype, hq, hkv, d, bs, lens, partition, seed, q_scale=1.0, scale=None):
+def run_decode(pa, dtype, hq, hkv, d, bs, lens, partition, seed, q_scale=1.0, scale=None, workspace=True):
     """Build the case through the library pool, run the kernel, return (gpu out, oracle out)."""
     from paged_kv_cache_341_b200.cache import PagedKVCache
     rng = np.random.default_rng(seed)
@@ -47,7 +47,7 @@ def run_decode(pa, dtype, hq, hkv, d, bs, lens, partition, seed, q_scale=1.0, sc
     q = q_host.cuda()
     out = torch.full((s, hq, d), float("nan"), dtype=TORCH[dtype], device="cuda")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    ws = pa.decode_workspace(s, hq, d, mb, bs, partition)
+    ws = pa.decode_workspace(s, hq, d, mb, bs, partition) if workspace else None
     cache.attend(q, out, scale, partition, ws)
     torch.cuda.synchronize()
     assert pa.pa_device_error() == 0
@@ -59,25 +59,54 @@ def run_decode(pa, dtype, hq, hkv, d, bs, lens, partition, seed, q_scale=1.0, sc
 LENS = [0, 1, 15, 16, 17, 100, 300]
 
 
+@pytest.fixture(params=["mma", "alu"])
+def path(request, monkeypatch):
+    """Consumer of 16-bit caches: tensor cores (default) or CUDA cores."""
+    if request.param == "alu":
+        monkeypatch.setenv("PA_DECODE_PATH", "alu")
+    else:
+        monkeypatch.delenv("PA_DECODE_PATH", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("hq,hkv", [(2, 2), (8, 4), (16, 4), (16, 2)])
 @pytest.mark.parametrize("bs", [16, 32])
 @pytest.mark.parametrize("partition", [0, 64])
-def test_decode_matches_oracle(pa, dtype, d, hq, hkv, bs, partition):
+def test_decode_matches_oracle(pa, path, dtype, d, hq, hkv, bs, partition):
+    if dtype == "f32" and path == "mma":
+        pytest.skip("float32 caches always take the CUDA-core consumer")
     gpu, ref, _, _ = run_decode(pa, dtype, hq, hkv, d, bs, LENS, partition, seed=hq * 7 + hkv + d + bs + partition)
-    assert_close(gpu, ref, dtype, "dtype=%s d=%d hq=%d hkv=%d bs=%d p=%d" % (dtype, d, hq, hkv, bs, partition))
+    assert_close(gpu, ref, dtype, "%s dtype=%s d=%d hq=%d hkv=%d bs=%d p=%d" % (path, dtype, d, hq, hkv, bs,
+                                                                             partition))
 
 
 @pytest.mark.parametrize("partition", [0, 512, 16])
-def test_many_units_per_cta(pa, partition):
+def test_many_units_per_cta(pa, path, partition):
     rng = np.random.default_rng(77)
     lens = [int(x) for x in rng.integers(1, 3000, size=300)] + [0, 1, 8192]
     gpu, ref, _, _ = run_decode(pa, "bf16", 32, 8, 128, 16, lens, partition, seed=9)
     assert_close(gpu, ref, "bf16", "p=%d" % partition)
 
 
-def test_single_token_returns_value_exactly(pa):
+def test_round_robin_without_workspace(pa, path):
+    """No workspace (single pass only): units dealt round-robin instead of by counter."""
+    rng = np.random.default_rng(78)
+    lens = [int(x) for x in rng.integers(1, 2500, size=200)] + [0, 1]
+    gpu, ref, _, _ = run_decode(pa, "bf16", 32, 8, 128, 16, lens, 0, seed=10, workspace=False)
+    assert_close(gpu, ref, "bf16", "round robin")
+
+
+@pytest.mark.parametrize("tile_heads", [1, 2, 4])
+def test_tile_heads_override(pa, path, monkeypatch, tile_heads):
+    monkeypatch.setenv("PA_DECODE_TILE_HEADS", str(tile_heads))
+    lens = [3, 16, 600, 1300]
+    gpu, ref, _, _ = run_decode(pa, "bf16", 32, 8, 128, 16, lens, 256, seed=31)
+    assert_close(gpu, ref, "bf16", "tile heads %d" % tile_heads)
+
+
+def test_single_token_returns_value_exactly(pa, path):
     for dtype in ("f32", "bf16", "f16"):
         gpu, ref, v_host, cache = run_decode(pa, dtype, 8, 2, 128, 16, [1, 1, 1], 0, seed=5, q_scale=10.0)
         for s in range(3):
@@ -90,7 +119,7 @@ def test_single_token_returns_value_exactly(pa):
         assert np.array_equal(gpu2, gpu)
 
 
-def test_zero_scale_and_large_scores(pa):
+def test_zero_scale_and_large_scores(pa, path):
     lens = [5, 33, 200]
     gpu, ref, _, _ = run_decode(pa, "f32", 4, 2, 64, 16, lens, 0, seed=11, scale=0.0)
     assert_close(gpu, ref, "f32", "scale=0")
@@ -100,7 +129,7 @@ def test_zero_scale_and_large_scores(pa):
     assert_close(gpu, ref, "bf16", "q x30")
 
 
-def test_split_matches_single_pass(pa):
+def test_split_matches_single_pass(pa, path):
     lens = [1, 40, 513, 1000, 2048]
     a, ref, _, _ = run_decode(pa, "bf16", 32, 8, 128, 16, lens, 0, seed=21)
     b, _, _, _ = run_decode(pa, "bf16", 32, 8, 128, 16, lens, 4096, seed=21)     # one partition each
