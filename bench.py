@@ -138,6 +138,20 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when not distributed)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_gbs(bytes_per_rank, ms_max, world):
+    """Whole-job throughput: every rank processed `bytes_per_rank` in at most `ms_max` ms."""
+    return world * bytes_per_rank / (ms_max / 1e3) / 1e9
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -335,10 +349,7 @@ def run_ours(args):
     clocks = sampler.stop() if sampler else None
     ms = t_start.elapsed_time(t_end) / args.steps
     att_ms = float(np.mean([a.elapsed_time(b) for a, b in att_ev]))
-    if world > 1:
-        t = torch.tensor([ms, att_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, att_ms = float(t[0]), float(t[1])
+    ms, att_ms = max_over_ranks([ms, att_ms], device="cuda")
     assert pa.pa_device_error() == 0
 
     # ---- end to end through the public API from pinned host memory
@@ -372,11 +383,8 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t[0])
-        e2e = {"value": round(world * e2e_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        e2e_ms = max_over_ranks([e2e_ms], device="cuda")[0]
+        e2e = {"value": round(whole_job_gbs(e2e_bytes, e2e_ms, world), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(in_bytes + meta_bytes + 8 * pairs_total / max(1, n_e2e)),
                "d2h_bytes_per_step": int(out.numel() * out.element_size()), "steps": n_e2e,
                "ms_per_step": round(e2e_ms / n_e2e, 4),
@@ -396,7 +404,7 @@ def run_ours(args):
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
-        value = world * kv_bytes / (ms / 1e3) / 1e9
+        value = whole_job_gbs(kv_bytes, ms, world)
         achieved = kv_bytes / (att_ms / 1e3) / 1e9
         traffic = traffic_record(w.name)
         line = {
@@ -409,8 +417,11 @@ def run_ours(args):
             "decode_tokens_per_s": round(world * sc.batch / (ms / 1e3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": "pa_decode_attention (decode_kernel + reduce_kernel), mean of %d launches; "
-                                   "peak = %s copy bandwidth" % (n_att, peak_kind),
+                         "kernel": "pa_decode_attention call (%s + reduce_kernel), mean of %d calls; "
+                                   "peak = %s copy bandwidth" % (
+                                       "decode_mma_kernel" if w.elem_bytes == 2 and
+                                       os.environ.get("PA_DECODE_PATH") != "alu" else "decode_kernel",
+                                       n_att, peak_kind),
                          "algorithmic_bytes_per_launch": kv_bytes},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,

@@ -79,9 +79,9 @@ def build(verbose=False):
 
 
 def kernel_digest():
-    """Digest of the decode kernel's sources (ties ncu counters to the code they were taken on)."""
+    """Digest of the decode kernel's sources and launch code (ties ncu counters to the code they were taken on)."""
     h = hashlib.sha256()
-    for name in ("decode.cuh", "ptx.cuh", "dtype.cuh"):
+    for name in ("decode.cuh", "ptx.cuh", "dtype.cuh", "pa_device.cu"):
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
