@@ -352,7 +352,11 @@ def run_ours(args):
     ms, att_ms = max_over_ranks([ms, att_ms], device="cuda")
     assert pa.pa_device_error() == 0
 
-    # ---- end to end through the public API from pinned host memory
+    # ---- end to end through the public API from pinned host memory.  Every
+    # step: host slot reservation, H2D of that step's q / new K,V (copy stream)
+    # and of slots / tables (compute stream), the kernels, D2H of the output.
+    # Inputs and outputs are double-buffered so step i's copies overlap step
+    # i-1's kernels; the host never waits for a step to finish.
     e2e = None
     if args.e2e_steps > 0:
         n_e2e = args.e2e_steps
@@ -360,26 +364,46 @@ def run_ours(args):
         for i in range(n_e2e):
             qi, ki, vi = sc.step_inputs(1 + i)
             host_in.append((qi.pin_memory(), ki.pin_memory(), vi.pin_memory()))
-        q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        copy_stream = torch.cuda.Stream()
+        dev_in = [(torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)) for _ in range(2)]
+        dev_out = [torch.empty_like(out) for _ in range(2)]
+        host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_read = [torch.cuda.Event() for _ in range(2)]
         in_bytes = q.numel() * q.element_size() + 2 * kn.numel() * kn.element_size()
-        meta_bytes = (c.d_tables.numel() + c.d_lens.numel()) * 4 + sc.batch * 8
+        meta_bytes = (c.d_tables[sc.rows].numel() + c.d_lens[sc.rows].numel()) * 4 + sc.batch * 8
+        ws_e2e = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
         e2e_bytes, pairs_total = 0, 0
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        copy_stream.wait_stream(stream)
         for i in range(n_e2e):
-            qi, ki, vi = host_in[i]
-            q_d.copy_(qi, non_blocking=True)
-            k_d.copy_(ki, non_blocking=True)
-            v_d.copy_(vi, non_blocking=True)
-            _, pr = c.decode_step(q_d, k_d, v_d, out, w.scale, part, ws_e2e(pa, sc, part), rows=sc.rows)
+            b = i % 2
+            qd, kd, vd = dev_in[b]
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(comp_done[b])
+                qi, ki, vi = host_in[i]
+                qd.copy_(qi, non_blocking=True)
+                kd.copy_(ki, non_blocking=True)
+                vd.copy_(vi, non_blocking=True)
+                in_ready[b].record(copy_stream)
+            stream.wait_event(in_ready[b])
+            if i >= 2:
+                stream.wait_event(out_read[b])
+            _, pr = c.decode_step(qd, kd, vd, dev_out[b], w.scale, part, ws_e2e, rows=sc.rows, stream=stream)
             pairs_total += pr.shape[0]
-            out_h.copy_(out, non_blocking=True)
-            stream.synchronize()
             e2e_bytes += sc.kv_bytes()
+            comp_done[b].record(stream)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(comp_done[b])
+                host_out[b].copy_(dev_out[b], non_blocking=True)
+                out_read[b].record(copy_stream)
+        stream.wait_stream(copy_stream)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -388,8 +412,9 @@ def run_ours(args):
                "h2d_bytes_per_step": int(in_bytes + meta_bytes + 8 * pairs_total / max(1, n_e2e)),
                "d2h_bytes_per_step": int(out.numel() * out.element_size()), "steps": n_e2e,
                "ms_per_step": round(e2e_ms / n_e2e, 4),
-               "note": "host slot reservation, pinned H2D of q/new K,V/slots/tables, kernels, D2H of out; "
-                       "sequences grow one token per step"}
+               "note": "per step: host slot reservation, pinned H2D of q/new K,V/slots/tables, kernels, "
+                       "D2H of out; copies overlap the previous step's kernels; sequences grow one token "
+                       "per step"}
         assert pa.pa_device_error() == 0
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N=1 only)
@@ -431,17 +456,6 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
-
-
-_WS = {}
-
-
-def ws_e2e(pa, sc, part):
-    key = id(sc)
-    if key not in _WS:
-        w, c = sc.w, sc.cache
-        _WS[key] = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
-    return _WS[key]
 
 
 def main():

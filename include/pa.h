@@ -180,13 +180,15 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *   partition_size 0: one pass over each whole context.  > 0 (a multiple of
  *                  block_size): split each context into partitions of
  *                  that many tokens, compute partial (max, sum, output) per
- *                  partition and merge them with a second kernel.
+ *                  partition and merge them with a second kernel (launched
+ *                  as a programmatic dependent of the first).
  *   workspace      device buffer of pa_decode_workspace_size() bytes, owned
  *                  by the caller; required when partition_size > 0.  With a
  *                  workspace the work units are handed out through a counter
- *                  in it (zeroed by a 4-byte memset on `stream` before each
- *                  launch); with NULL (only when partition_size == 0) they are
- *                  dealt round-robin.  Calls sharing a workspace must not
+ *                  in it; the counter is zeroed
+ *                  by a cudaMemsetAsync on `stream` before each launch.  With
+ *                  NULL (only when partition_size == 0) the units are dealt
+ *                  round-robin.  Calls sharing a workspace must not
  *                  overlap on the GPU.
  * Supported: head_dim 64 or 128; Hq/Hkv in {1,2,4,8}; block_size a multiple
  * of 16; dtype f32/f16/bf16.  Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED,

@@ -40,8 +40,12 @@
 //   the final division by l cancels the choice of m exactly, so accumulator
 //   rescaling is rare.
 // * With partitions, each unit writes its (m, l, unnormalised output) in
-//   float32 and reduce_kernel merges them; sequences that fit in one
-//   partition are written out directly.
+//   float32 and reduce_kernel merges them; it is launched as a programmatic
+//   dependent of the decode kernel, so its CTAs are resident before the
+//   decode grid drains and start the moment its writes are visible.
+//   Sequences that fit in one partition are written out directly.  (Merging
+//   inside the decode kernel -- the last partition of a head merges -- was
+//   measured 8 % slower: the merging warp stalls its CTA's pipeline.)
 #ifndef PAGEDATTN_DECODE_CUH
 #define PAGEDATTN_DECODE_CUH
 
@@ -413,6 +417,7 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) pl.init();
   __syncthreads();
+  allow_dependent_launch();
 
   if (warp == HT) {
     run_producer<T, D, G, false>(pl, prm, &tm_k, &tm_v, lane);
@@ -666,6 +671,7 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) pl.init();
   __syncthreads();
+  allow_dependent_launch();
 
   if (warp == HT) {
     run_producer<T, D, G, true>(pl, prm, &tm_k, &tm_v, lane);
@@ -857,7 +863,9 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
 // Merge of per-partition partials: M = max m_p, w_p = 2^(m_p - M),
 // out = sum_p w_p acc_p / sum_p w_p l_p.  One warp per (sequence, query
 // head); sequences that fit one partition were written by the decode kernel
-// and are skipped.
+// and are skipped.  Launched as a programmatic dependent of the decode kernel:
+// it waits (griddepcontrol.wait) until that grid has finished and its writes
+// are visible before reading anything it wrote.
 // ===========================================================================
 struct ReduceParams {
   const int32_t* context_lens;
@@ -874,14 +882,16 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   constexpr int PER = D / 32;                // contiguous elements per lane
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
   const int s = blockIdx.y;
-  int len = prm.context_lens[s];
+  int len = prm.context_lens[s];             // written before the decode launch: safe to read now
   len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
   const int np = parts_of(len, prm.partition_size);
+  wait_prerequisite_grids();
   if (np <= 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hq = blockIdx.x * kReduceWarps + warp;
   if (hq >= prm.num_q_heads) return;
   const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + hq) * prm.max_parts;
+  // lane p holds partition p's (m, l) (partitions beyond 32 fold into lanes)
   float mx = -INFINITY;
   for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
 #pragma unroll
@@ -900,8 +910,23 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
     const int pl = p0 + lane;
     const float wl = pl < np ? exp2_approx(prm.part_ml[base + pl].x - mx) : 0.f;
     const int n = min(32, np - p0);
-#pragma unroll 4
-    for (int k = 0; k < n; ++k) {
+    int k = 0;
+    for (; k + 4 <= n; k += 4) {            // four partitions' loads in flight at once
+      float2 v[4][PER / 2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + k + u) * D + lane * PER);
+#pragma unroll
+        for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wl, k + u);
+#pragma unroll
+        for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(w, w), v[u][e]);
+      }
+    }
+    for (; k < n; ++k) {
       const float w = __shfl_sync(0xffffffffu, wl, k);
       const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + k) * D + lane * PER);
 #pragma unroll

@@ -226,6 +226,7 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.qk_scale = a.scale * 1.4426950408889634f;
 
   if (prm.sched) {
+    // the unit counter starts at zero on every launch
     e = cudaMemsetAsync(prm.sched, 0, sizeof(int), a.stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(unit counter)");
   }
@@ -244,11 +245,21 @@ pa_status launch_decode(const DecodeArgs& a) {
     rp.partition_size = a.P;
     rp.max_parts = np;
     rp.cap = a.max_blocks * a.BS;
-    const dim3 rgrid((a.Hq + pa::kReduceWarps - 1) / pa::kReduceWarps, a.S);
-    pa::reduce_kernel<T, D><<<rgrid, pa::kReduceWarps * 32, 0, a.stream>>>(rp);
-    e = cudaGetLastError();
+    // programmatic dependent launch: resident early, waits for the decode grid
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((a.Hq + pa::kReduceWarps - 1) / pa::kReduceWarps, a.S);
+    cfg.blockDim = dim3(pa::kReduceWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, D>, rp);
     if (e != cudaSuccess) return cuda_fail(e, "reduce_kernel launch");
   }
+
   return pa::ok();
 }
 

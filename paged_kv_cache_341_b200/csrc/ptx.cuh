@@ -156,6 +156,16 @@ __device__ __forceinline__ void fmul2(float2& d, const float2 s) {
       : "f"(s.x), "f"(s.y));
 }
 
+// Programmatic dependent launch: let the next kernel on the stream launch now
+// (its CTAs start and then wait), and, in that kernel, wait until the
+// prerequisite grid has completed and its memory operations are visible.
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_prerequisite_grids() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // 2^x with the hardware approximation (ex2.approx; 2^0 = 1 and 2^-inf = 0 exactly).
 __device__ __forceinline__ float exp2_approx(float x) {
   float y;
