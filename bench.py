@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3_8b_gqa")
     ap.add_argument("--partition", type=int, default=None, help="override the workload's partition size")
+    ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -196,7 +197,7 @@ def run_reference(args):
     world, rank, _ = dist_setup()
     if rank != 0:
         return
-    sc = ReferenceScenario(args.workload)
+    sc = ReferenceScenario(args.workload, args.block_size)
     q_host, _, _ = sc.step_inputs(0)
     per_step_budget = max(0.002, 90.0 / (args.steps + args.warmup))
     seqs = pick_sample(sc, per_step_budget, q_host)
@@ -224,10 +225,10 @@ def run_reference(args):
 class ReferenceScenario:
     """The workload on the host only (no GPU): tables from the oracle pool, values from the generator."""
 
-    def __init__(self, name):
+    def __init__(self, name, block_size=None):
         from oracle import OraclePool
         from paged_kv_cache_341_b200 import workloads
-        w = workloads.get(name)
+        w = workloads.get(name, block_size)
         self.w = w
         self.lens0 = workloads.lengths(w)
         op = OraclePool(w.num_blocks, w.block_size, workloads.pool_order(w.num_blocks, w.seed))
@@ -276,6 +277,7 @@ def workload_config(sc, args):
             "head_dim": w.head_dim, "block_size": w.block_size, "cache_dtype": w.dtype,
             "mean_context": round(float(np.mean(lens)), 1), "max_context": int(np.max(lens)),
             "partition_size": p, "num_blocks": w.num_blocks, "layers": 1,
+            "slot_waste": round(sc.slot_waste(), 5) if hasattr(sc, "slot_waste") else None,
             "l2": "inputs larger than L2 (K/V set %.2f GB vs 126 MB L2), no flush" % (
                 int(np.sum(lens)) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes / 1e9),
             "parallelism": "replicas x%d (weak)" % args.gpus}
@@ -292,7 +294,7 @@ def run_ours(args):
     build.ensure_built()
     from paged_kv_cache_341_b200.scenarios import Scenario
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-    sc = Scenario(args.workload, keep_host=want_cpu)
+    sc = Scenario(args.workload, keep_host=want_cpu, block_size=args.block_size)
     w, c = sc.w, sc.cache
     part = w.partition_size if args.partition is None else args.partition
     stream = torch.cuda.current_stream()

@@ -178,7 +178,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *                  tokens < context_lens[s] must be valid block ids
  *   context_lens:  device int32 [S], each <= max_blocks_per_seq*block_size
  *   partition_size 0: one pass over each whole context.  > 0 (a multiple of
- *                  block_size): split each context into partitions of
+ *                  block_size and of 16): split each context into partitions of
  *                  that many tokens, compute partial (max, sum, output) per
  *                  partition and merge them with a second kernel (launched
  *                  as a programmatic dependent of the first).
@@ -191,7 +191,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *                  round-robin.  Calls sharing a workspace must not
  *                  overlap on the GPU.
  * Supported: head_dim 64 or 128; Hq/Hkv in {1,2,4,8}; block_size a multiple
- * of 16; dtype f32/f16/bf16.  Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED,
+ * of 16, or 8; dtype f32/f16/bf16.  Errors: PA_ERR_INVALID, PA_ERR_UNSUPPORTED,
  * PA_ERR_CUDA. */
 pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_cache,
                               int32_t num_blocks, const int32_t* block_tables,

@@ -281,10 +281,17 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
     for (int c = 0; c < nchunks; ++c) {
       const int tok = tok_begin + c * kChunkTokens;
       const int ntok = max(0, min(kChunkTokens, tok_end - tok));
-      int phys = 0, within = 0;
-      if (ntok > 0) {
-        const int blk = tok / BS;
-        within = tok - blk * BS;
+      // A chunk is one 16-row piece of one block, or, with 8-token blocks,
+      // two 8-row pieces of two logically consecutive blocks.
+      const int piece_rows = BS < kChunkTokens ? BS : kChunkTokens;
+      const int npieces = kChunkTokens / piece_rows;
+      int rows[2] = {0, 0};
+      int loaded = 0;
+      for (int pc = 0; pc < npieces; ++pc) {
+        const int t0 = tok + pc * piece_rows;
+        if (t0 >= tok_end) break;
+        const int blk = t0 / BS;
+        const int within = t0 - blk * BS;
         const int wb = blk & ~31;
         if (seq != tw_seq || wb != tw_base) {
           tw_seq = seq;
@@ -292,11 +299,13 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
           const int idx = wb + lane;
           tw_val = idx < MB ? prm.block_tables[static_cast<size_t>(seq) * MB + idx] : 0;
         }
-        phys = __shfl_sync(0xffffffffu, tw_val, blk - wb);
+        int phys = __shfl_sync(0xffffffffu, tw_val, blk - wb);
         if (phys < 0 || phys >= prm.num_blocks) {
           if (lane == 0) set_device_error(DEVERR_BAD_BLOCK_ID);
           phys = 0;
         }
+        rows[pc] = phys * BS + within;
+        loaded = pc + 1;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag))) {
         ok = false;
@@ -313,30 +322,33 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
         m.qslot = qslot;
         m.pad = 0;
         pl.meta[stage] = m;
-        if (ntok > 0) {
-          mbar_arrive_expect_tx(&pl.full[stage], 2 * prm.tile_bytes);
+        if (loaded > 0) {
+          mbar_arrive_expect_tx(&pl.full[stage], 2 * prm.tile_bytes / npieces * loaded);
         } else {
           mbar_arrive(&pl.full[stage]);
         }
       }
       __syncwarp();
-      if (ntok > 0) {
-        const int row = phys * BS + within;
+      if (loaded > 0) {
         T* dk = pl.s_k + stage * pl.tile_elems;
         T* dv = pl.s_v + stage * pl.tile_elems;
         if constexpr (kSwizzled) {
-          // lanes split the 2 * HT * kHalves boxes of this stage
+          // lanes split the loaded pieces' K and V boxes, one per (head, column block)
           const int nbox = HT * kHalves;
-          for (int b = lane; b < 2 * nbox; b += 32) {
-            const int kv = b >= nbox ? 1 : 0;
-            const int hb = b - kv * nbox;                 // head-in-tile * kHalves + column block
-            T* dst = (kv ? dv : dk) + hb * kChunkTokens * kBoxElems;
-            tma_load_3d(dst, kv ? tm_v : tm_k, &pl.full[stage], 0, tile * HT * kHalves + hb, row, policy);
+          for (int b = lane; b < loaded * 2 * nbox; b += 32) {
+            const int pc = b / (2 * nbox);
+            const int r = b - pc * 2 * nbox;
+            const int kv = r >= nbox ? 1 : 0;
+            const int hb = r - kv * nbox;                 // head-in-tile * kHalves + column block
+            T* dst = (kv ? dv : dk) + hb * kChunkTokens * kBoxElems + pc * piece_rows * kBoxElems;
+            tma_load_3d(dst, kv ? tm_v : tm_k, &pl.full[stage], 0, tile * HT * kHalves + hb, rows[pc], policy);
           }
         } else {
-          if (lane == 0) {
-            tma_load_3d(dk, tm_k, &pl.full[stage], 0, tile * HT, row, policy);
-            tma_load_3d(dv, tm_v, &pl.full[stage], 0, tile * HT, row, policy);
+          if (lane < 2 * loaded) {
+            const int pc = lane >> 1;
+            const int kv = lane & 1;
+            T* dst = (kv ? dv : dk) + pc * piece_rows * HT * D;
+            tma_load_3d(dst, kv ? tm_v : tm_k, &pl.full[stage], 0, tile * HT, rows[pc], policy);
           }
         }
       }

@@ -110,7 +110,7 @@ CUtensorMapDataType map_type<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_B
 // 16 tokens x one column block, stored 128B-swizzled in shared memory.
 template <typename T>
 pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, long long rows, int tile_heads,
-                         bool swizzled) {
+                         bool swizzled, int box_rows) {
   auto encode = tensor_map_encoder();
   if (!encode) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t row_bytes = static_cast<cuuint64_t>(Hkv) * D * sizeof(T);
@@ -121,7 +121,7 @@ pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, lon
     const cuuint64_t dims[3] = {box_elems, static_cast<cuuint64_t>(Hkv) * D / box_elems,
                                 static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pa::kSwizzleBytes), row_bytes};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_elems), 1, static_cast<cuuint32_t>(pa::kChunkTokens)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_elems), 1, static_cast<cuuint32_t>(box_rows)};
     r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -130,7 +130,7 @@ pa_status make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, lon
                                 static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * sizeof(T), row_bytes};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(tile_heads),
-                               static_cast<cuuint32_t>(pa::kChunkTokens)};
+                               static_cast<cuuint32_t>(box_rows)};
     r = encode(map, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, elem_strides,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -194,9 +194,10 @@ pa_status launch_decode(const DecodeArgs& a) {
 
   CUtensorMap tm_k, tm_v;
   const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
-  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, ht, mma);
+  const int box_rows = a.BS < pa::kChunkTokens ? a.BS : pa::kChunkTokens;
+  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, ht, mma, box_rows);
   if (st != PA_OK) return st;
-  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, ht, mma);
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, ht, mma, box_rows);
   if (st != PA_OK) return st;
 
   pa::DecodeParams prm;
@@ -351,13 +352,15 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: need Hq a positive multiple of Hkv");
   if (num_blocks <= 0 || max_blocks_per_seq <= 0 || block_size <= 0)
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: bad pool sizes");
-  if (block_size % pa::kChunkTokens != 0)
-    return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: block_size must be a multiple of 16");
+  if (block_size != 8 && block_size % pa::kChunkTokens != 0)
+    return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: block_size must be 8 or a multiple of 16");
   if (static_cast<long long>(num_blocks) * block_size >= (1ll << 31) ||
       static_cast<long long>(max_blocks_per_seq) * block_size >= (1ll << 31))
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: pool or table too large for 32-bit token indices");
-  if (partition_size < 0 || (partition_size > 0 && partition_size % block_size != 0))
-    return pa::fail(PA_ERR_INVALID, "pa_decode_attention: partition_size must be 0 or a multiple of block_size");
+  if (partition_size < 0 ||
+      (partition_size > 0 && (partition_size % block_size != 0 || partition_size % pa::kChunkTokens != 0)))
+    return pa::fail(PA_ERR_INVALID,
+                    "pa_decode_attention: partition_size must be 0 or a multiple of block_size and of 16");
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
     return pa::fail(PA_ERR_INVALID, "pa_decode_attention: scale must be finite");
   if (num_seqs == 0) return pa::ok();

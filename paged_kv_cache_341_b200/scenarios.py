@@ -17,8 +17,8 @@ from .cache import PagedKVCache
 
 
 class Scenario:
-    def __init__(self, name, device="cuda", fill_values=True, keep_host=False):
-        w = workloads.get(name)
+    def __init__(self, name, device="cuda", fill_values=True, keep_host=False, block_size=None):
+        w = workloads.get(name, block_size)
         self.w = w
         self.lens0 = workloads.lengths(w)
         order = workloads.pool_order(w.num_blocks, w.seed)
@@ -74,6 +74,13 @@ class Scenario:
         w = self.w
         lens = self.cache.lens[self.rows].astype(np.int64)
         return int(lens.sum()) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+
+    def slot_waste(self):
+        """Fraction of allocated token slots left empty in the batch's blocks (tail waste)."""
+        w = self.w
+        lens = self.cache.lens[self.rows].astype(np.int64)
+        blocks = (-(-lens // w.block_size)).sum()
+        return float(1.0 - lens.sum() / (blocks * w.block_size))
 
     def unique_kv_bytes(self):
         """Distinct K/V bytes behind the batch (shared blocks counted once)."""

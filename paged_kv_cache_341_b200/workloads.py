@@ -78,8 +78,12 @@ WORKLOADS = {
 }
 
 
-def get(name):
-    return dataclasses.replace(WORKLOADS[name])
+def get(name, block_size=None):
+    """A copy of workload ``name``; ``block_size`` overrides its block size (block-size sweeps)."""
+    w = dataclasses.replace(WORKLOADS[name])
+    if block_size is not None:
+        w.block_size = int(block_size)
+    return w
 
 
 def lengths(w):

@@ -54,7 +54,7 @@ def test_decode_rejects_bad_arguments_on_host(built_library):
                                        a["out"], a["dt"], a["stream"])
 
     assert call(hq=3, hkv=2) == pa.PA_ERR_INVALID
-    assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
+    assert call(bs=24) == pa.PA_ERR_UNSUPPORTED
     assert call(p=24) == pa.PA_ERR_INVALID                  # not a multiple of block_size
     assert call(p=32) == pa.PA_ERR_INVALID                  # workspace missing
     assert call(dt=7) == pa.PA_ERR_INVALID

@@ -72,7 +72,7 @@ def path(request, monkeypatch):
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("hq,hkv", [(2, 2), (8, 4), (16, 4), (16, 2)])
-@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("bs", [8, 16, 32])
 @pytest.mark.parametrize("partition", [0, 64])
 def test_decode_matches_oracle(pa, path, dtype, d, hq, hkv, bs, partition):
     if dtype == "f32" and path == "mma":
