@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_gqa")
     ap.add_argument("--partition", type=int, default=None, help="override the workload's partition size")
     ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared-prefix workload: attend the shared prefix once for all sequences "
+                         "(pa_decode_attention_shared_prefix)")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -313,13 +316,31 @@ def run_ours(args):
     kv_bytes = sc.kv_bytes()
     config = workload_config(sc, args)
     launches_per_step = (1 if pairs.shape[0] else 0) + 1 + (2 if part > 0 else 1)
+    cascade = args.cascade and w.shared_prefix > 0
+    if cascade:
+        pblocks = w.shared_prefix // w.block_size
+        prefix_ids = c.d_tables[sc.rows.start, :pblocks].contiguous()
+        suffix_tables = c.d_tables[sc.rows, pblocks:]
+        suffix_lens = (lens - w.shared_prefix).contiguous()
+        ws = torch.empty(pa.pa_shared_prefix_workspace_size(sc.batch, w.num_q_heads, w.head_dim, w.shared_prefix,
+                                                            suffix_tables.shape[1], w.block_size, part),
+                         dtype=torch.uint8, device="cuda")
+        launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 3
+        config["cascade"] = {"prefix_tokens": w.shared_prefix, "unique_kv_bytes": sc.unique_kv_bytes()}
+
+    def attend():
+        if cascade:
+            pa.pa_decode_attention_shared_prefix(q, c.k_cache, c.v_cache, prefix_ids, w.shared_prefix,
+                                                 suffix_tables, suffix_lens, w.scale, out, part, ws)
+        else:
+            c.attend(q, out, w.scale, part, ws, tables=tables, lens=lens)
 
     def step(ev0=None, ev1=None):
         c.copy_blocks(d_pairs)
         c.append(kn, vn, d_slots)
         if ev0 is not None:
             ev0.record(stream)
-        c.attend(q, out, w.scale, part, ws, tables=tables, lens=lens)
+        attend()
         if ev1 is not None:
             ev1.record(stream)
 

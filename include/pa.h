@@ -201,6 +201,44 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
                               int32_t partition_size, void* workspace, size_t workspace_bytes,
                               void* out, pa_dtype dtype, void* stream);
 
+/* Bytes of device workspace pa_decode_attention_shared_prefix takes: 256
+ * bytes for the work-unit counter plus one float32 partial (max, sum, D
+ * values) per (sequence, query head, part), where the parts are the prefix's
+ * ceil(prefix_len / 1024) slices followed by the suffix's partitions
+ * (ceil(max_suffix_blocks * block_size / partition_size), or 1 when
+ * partition_size == 0).  0 for invalid sizes. */
+size_t pa_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                       int32_t prefix_len, int32_t max_suffix_blocks,
+                                       int32_t block_size, int32_t partition_size);
+
+/* Decode attention when every sequence starts with the same prefix blocks
+ * (a system prompt shared copy-on-write by many sequences: "Paged Attention",
+ * aidolsgroup.com, section "Example"; agentechip.com "Shared Prefix
+ * Caching").  The result equals pa_decode_attention with, for sequence s,
+ * block table prefix_blocks ++ suffix_tables[s] and context length
+ * prefix_len + suffix_lens[s].  The prefix is attended once per KV head for
+ * all S*G query rows together on the tensor cores (each prefix K/V tile read
+ * once per 64 query rows), the suffixes by the decode kernel, and one merge
+ * combines the partial results.
+ *
+ *   prefix_blocks  device int32 [prefix_len / block_size]
+ *   prefix_len     tokens; a multiple of block_size and of 16 (0: plain call)
+ *   suffix_tables  device int32 rows of max_suffix_blocks valid entries,
+ *                  suffix_table_stride elements apart (>= max_suffix_blocks)
+ *   suffix_lens    device int32 [S], each <= max_suffix_blocks*block_size
+ *   workspace      pa_shared_prefix_workspace_size() bytes, caller-owned
+ * Other arguments as for pa_decode_attention.  f16/bf16 caches only
+ * (PA_ERR_UNSUPPORTED otherwise). */
+pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                            int32_t num_blocks, const int32_t* prefix_blocks,
+                                            int32_t prefix_len, const int32_t* suffix_tables,
+                                            int32_t suffix_table_stride, int32_t max_suffix_blocks,
+                                            const int32_t* suffix_lens, int32_t num_seqs,
+                                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                            int32_t block_size, float scale, int32_t partition_size,
+                                            void* workspace, size_t workspace_bytes, void* out,
+                                            pa_dtype dtype, void* stream);
+
 /* Largest workspace pa_decode_attention_static can use: 32 MiB. */
 #define PA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
 

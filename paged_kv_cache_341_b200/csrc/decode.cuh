@@ -71,6 +71,9 @@ struct DecodeParams {
   float* part_acc;               // [S][Hq][NP][D]   (partitioned mode)
   float2* part_ml;               // [S][Hq][NP]      (m in base-2 units, l)
   int* sched;                    // unit counter (zeroed before launch), or null: static order
+  int table_stride;              // elements between rows of block_tables (>= max_blocks)
+  int part_offset;               // partial index of partition 0 (shared-prefix mode)
+  int force_partials;            // write partials even for single-partition sequences
   int num_seqs, num_q_heads, num_kv_heads;
   int max_blocks, block_size, num_blocks;
   int partition_size;            // 0 = whole context in one unit
@@ -297,7 +300,7 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
           tw_seq = seq;
           tw_base = wb;
           const int idx = wb + lane;
-          tw_val = idx < MB ? prm.block_tables[static_cast<size_t>(seq) * MB + idx] : 0;
+          tw_val = idx < MB ? prm.block_tables[static_cast<size_t>(seq) * prm.table_stride + idx] : 0;
         }
         int phys = __shfl_sync(0xffffffffu, tw_val, blk - wb);
         if (phys < 0 || phys >= prm.num_blocks) {
@@ -558,7 +561,7 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
       for (int g = 0; g < G; ++g) {
         if (g % NG != grp) continue;
         const int hq = hq0 + g;
-        if (mt.nparts == 1) {
+        if (mt.nparts == 1 && !prm.force_partials) {
           const float inv = l[g] > 0.f ? 1.0f / l[g] : 0.f;
           T* orow = static_cast<T*>(prm.out) + (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq) * D;
 #pragma unroll
@@ -572,7 +575,8 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
             Chunk<T>::store(orow + (li + k * L) * EPC, o);
           }
         } else {
-          const size_t pidx = (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq) * prm.max_parts + mt.part;
+          const size_t pidx =
+              (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq) * prm.max_parts + prm.part_offset + mt.part;
           float* prow = prm.part_acc + pidx * D;
 #pragma unroll
           for (int k = 0; k < NCH; ++k) {
@@ -827,7 +831,7 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
       }
       const int hq0 = (mt.tile * HT + j) * G;
       const bool w0 = h0 < G, w1 = h0 + 1 < G;
-      if (mt.nparts == 1) {
+      if (mt.nparts == 1 && !prm.force_partials) {
         const float i0 = l0 > 0.f ? 1.0f / l0 : 0.f;
         const float i1 = l1 > 0.f ? 1.0f / l1 : 0.f;
         T* r0 = static_cast<T*>(prm.out) + (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq0 + h0) * D;
@@ -845,7 +849,8 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
           }
         }
       } else {
-        const size_t p0 = (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq0 + h0) * prm.max_parts + mt.part;
+        const size_t p0 =
+            (static_cast<size_t>(mt.seq) * prm.num_q_heads + hq0 + h0) * prm.max_parts + prm.part_offset + mt.part;
         const size_t p1 = p0 + prm.max_parts;
         float* r0 = prm.part_acc + p0 * D;
         float* r1 = prm.part_acc + p1 * D;
@@ -885,6 +890,7 @@ struct ReduceParams {
   const float2* part_ml;
   void* out;
   int num_seqs, num_q_heads, partition_size, max_parts, cap;
+  int part_offset;               // partials before partition 0 (shared-prefix splits); 0 otherwise
 };
 
 constexpr int kReduceWarps = 8;
@@ -896,9 +902,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   const int s = blockIdx.y;
   int len = prm.context_lens[s];             // written before the decode launch: safe to read now
   len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
-  const int np = parts_of(len, prm.partition_size);
+  const int np = prm.part_offset + parts_of(len, prm.partition_size);
   wait_prerequisite_grids();
-  if (np <= 1) return;
+  if (prm.part_offset == 0 && np <= 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hq = blockIdx.x * kReduceWarps + warp;
   if (hq >= prm.num_q_heads) return;
@@ -908,6 +914,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (mx == -INFINITY) mx = 0.f;            // no partition saw a token: all weights are 0
   float lsum = 0.f;
   for (int p = lane; p < np; p += 32) {
     const float2 ml = prm.part_ml[base + p];
@@ -945,7 +952,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
       for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(w, w), src[e]);
     }
   }
-  const float inv = 1.0f / lsum;
+  const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
   T* dst = static_cast<T*>(prm.out) + (static_cast<size_t>(s) * prm.num_q_heads + hq) * D + lane * PER;
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) {

@@ -12,6 +12,7 @@
 
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "prefix.cuh"
 #include "pa.h"
 #include "pa_common.h"
 
@@ -85,6 +86,10 @@ struct DecodeArgs {
   void* out;
   pa_dtype dtype;
   cudaStream_t stream;
+  // shared-prefix mode (pa_decode_attention_shared_prefix); plain calls leave the defaults
+  int table_stride = 0;          // 0: rows of block_tables are max_blocks apart
+  int part_offset = 0;           // partials before partition 0 (prefix splits)
+  int total_parts = 0;           // 0: ceil(max_blocks*block_size/P), else the partial row stride
 };
 
 constexpr size_t kSchedBytes = 256;   // unit counter at the head of the workspace
@@ -187,7 +192,8 @@ pa_status launch_decode(const DecodeArgs& a) {
   if (per_sm < 1) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: kernel does not fit on an SM");
 
   const int n_tiles = a.Hkv / ht;
-  const int np = max_parts(a.max_blocks, a.BS, a.P);
+  const int np = a.total_parts > 0 ? a.total_parts : max_parts(a.max_blocks, a.BS, a.P);
+  const bool partials = a.P > 0 || a.part_offset > 0;
   const long long units_bound = static_cast<long long>(a.S) * n_tiles * np;
   const long long slots = static_cast<long long>(dev.sms) * per_sm;
   const int grid = static_cast<int>(units_bound < slots ? units_bound : slots);
@@ -209,8 +215,11 @@ pa_status launch_decode(const DecodeArgs& a) {
   const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
   char* ws = static_cast<char*>(a.workspace);
   prm.sched = ws ? reinterpret_cast<int*>(ws) : nullptr;
-  prm.part_acc = a.P > 0 ? reinterpret_cast<float*>(ws + kSchedBytes) : nullptr;
-  prm.part_ml = a.P > 0 ? reinterpret_cast<float2*>(prm.part_acc + acc_elems) : nullptr;
+  prm.part_acc = partials ? reinterpret_cast<float*>(ws + kSchedBytes) : nullptr;
+  prm.part_ml = partials ? reinterpret_cast<float2*>(prm.part_acc + acc_elems) : nullptr;
+  prm.table_stride = a.table_stride > 0 ? a.table_stride : a.max_blocks;
+  prm.part_offset = a.part_offset;
+  prm.force_partials = a.part_offset > 0 ? 1 : 0;
   prm.num_seqs = a.S;
   prm.num_q_heads = a.Hq;
   prm.num_kv_heads = a.Hkv;
@@ -235,7 +244,7 @@ pa_status launch_decode(const DecodeArgs& a) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_kernel launch");
 
-  if (a.P > 0) {
+  if (partials) {
     pa::ReduceParams rp;
     rp.context_lens = a.context_lens;
     rp.part_acc = prm.part_acc;
@@ -246,6 +255,7 @@ pa_status launch_decode(const DecodeArgs& a) {
     rp.partition_size = a.P;
     rp.max_parts = np;
     rp.cap = a.max_blocks * a.BS;
+    rp.part_offset = a.part_offset;
     // programmatic dependent launch: resident early, waits for the decode grid
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((a.Hq + pa::kReduceWarps - 1) / pa::kReduceWarps, a.S);
@@ -281,6 +291,88 @@ pa_status dispatch_dim(const DecodeArgs& a) {
     case 64: return dispatch_group<T, 64>(a);
     case 128: return dispatch_group<T, 128>(a);
     default: return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: head_dim must be 64 or 128");
+  }
+}
+
+// Split of the shared prefix into slices of this many tokens (one CTA per
+// slice, 64 query rows and one KV head); fixed so that the workspace size is a
+// function of the arguments alone.
+constexpr int kPrefixSplitTokens = 1024;
+
+int prefix_splits(int prefix_len) { return (prefix_len + kPrefixSplitTokens - 1) / kPrefixSplitTokens; }
+
+struct PrefixArgs {
+  const int32_t* prefix_blocks;
+  int prefix_len;
+};
+
+template <typename T, int D, int G>
+pa_status launch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
+  DeviceInfo dev;
+  pa_status st = device_info(&dev);
+  if (st != PA_OK) return st;
+  const size_t stage_bytes = static_cast<size_t>(pa::kPrefixTile) * D * sizeof(T);
+  int stages = 3;
+  const int forced_st = env_int("PA_PREFIX_STAGES");
+  if (forced_st >= 2 && forced_st <= 8) stages = forced_st;
+  while (stages >= 2 && pa::prefix_smem_bytes(stages, stage_bytes) > static_cast<size_t>(dev.smem_optin)) --stages;
+  if (stages < 2) return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: stage does not fit in shared memory");
+  const size_t smem = pa::prefix_smem_bytes(stages, stage_bytes);
+  auto kern = pa::prefix_attention_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix)");
+
+  CUtensorMap tm_k, tm_v;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
+  const int box_rows = a.BS < pa::kChunkTokens ? a.BS : pa::kChunkTokens;
+  st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+
+  const int np = a.total_parts;
+  const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
+  char* ws = static_cast<char*>(a.workspace);
+  pa::PrefixParams prm;
+  prm.q = a.q;
+  prm.prefix_blocks = pf.prefix_blocks;
+  prm.part_acc = reinterpret_cast<float*>(ws + kSchedBytes);
+  prm.part_ml = reinterpret_cast<float2*>(prm.part_acc + acc_elems);
+  prm.num_seqs = a.S;
+  prm.num_q_heads = a.Hq;
+  prm.num_kv_heads = a.Hkv;
+  prm.block_size = a.BS;
+  prm.num_blocks = a.num_blocks;
+  prm.prefix_len = pf.prefix_len;
+  prm.split_tokens = kPrefixSplitTokens;
+  prm.max_parts = np;
+  prm.stages = stages;
+  prm.stage_bytes = static_cast<uint32_t>(stage_bytes);
+  prm.qk_scale = a.scale * 1.4426950408889634f;
+  const dim3 grid((a.S * G + pa::kPrefixRows - 1) / pa::kPrefixRows, a.Hkv, prefix_splits(pf.prefix_len));
+  kern<<<grid, (pa::kPrefixWarps + 1) * 32, smem, a.stream>>>(tm_k, tm_v, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefix_attention_kernel launch");
+  return PA_OK;
+}
+
+template <typename T, int D>
+pa_status dispatch_prefix_group(const DecodeArgs& a, const PrefixArgs& pf) {
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_prefix<T, D, 1>(a, pf);
+    case 2: return launch_prefix<T, D, 2>(a, pf);
+    case 4: return launch_prefix<T, D, 4>(a, pf);
+    case 8: return launch_prefix<T, D, 8>(a, pf);
+    default: return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: Hq/Hkv must be 1, 2, 4 or 8");
+  }
+}
+
+template <typename T>
+pa_status dispatch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
+  switch (a.D) {
+    case 64: return dispatch_prefix_group<T, 64>(a, pf);
+    case 128: return dispatch_prefix_group<T, 128>(a, pf);
+    default: return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: head_dim must be 64 or 128");
   }
 }
 
@@ -439,6 +531,69 @@ pa_status pa_decode_attention_static(const void* q, const void* k_cache, const v
   return pa_decode_attention(q, k_cache, v_cache, num_blocks, block_tables, max_blocks_per_seq, context_lens,
                              num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale, partition_size, ws,
                              ws ? PA_STATIC_WORKSPACE_BYTES : 0, out, dtype, stream);
+}
+
+size_t pa_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t prefix_len,
+                                       int32_t max_suffix_blocks, int32_t block_size, int32_t partition_size) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || prefix_len < 0 || max_suffix_blocks <= 0 ||
+      block_size <= 0 || partition_size < 0)
+    return 0;
+  const size_t np = static_cast<size_t>(prefix_splits(prefix_len)) +
+                    static_cast<size_t>(max_parts(max_suffix_blocks, block_size, partition_size));
+  return kSchedBytes + static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
+}
+
+pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                            int32_t num_blocks, const int32_t* prefix_blocks, int32_t prefix_len,
+                                            const int32_t* suffix_tables, int32_t suffix_table_stride,
+                                            int32_t max_suffix_blocks, const int32_t* suffix_lens, int32_t num_seqs,
+                                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                            int32_t block_size, float scale, int32_t partition_size,
+                                            void* workspace, size_t workspace_bytes, void* out, pa_dtype dtype,
+                                            void* stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: the tensor-core path takes f16/bf16 caches");
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return pa::fail(PA_ERR_INVALID, "shared prefix: need Hq a positive multiple of Hkv");
+  if (num_blocks <= 0 || max_suffix_blocks <= 0 || block_size <= 0 || suffix_table_stride < max_suffix_blocks)
+    return pa::fail(PA_ERR_INVALID, "shared prefix: bad pool or table sizes");
+  if (block_size != 8 && block_size % pa::kChunkTokens != 0)
+    return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: block_size must be 8 or a multiple of 16");
+  if (prefix_len < 0 || prefix_len % block_size != 0 || prefix_len % pa::kChunkTokens != 0)
+    return pa::fail(PA_ERR_INVALID, "shared prefix: prefix_len must be a multiple of block_size and of 16");
+  if (static_cast<long long>(num_blocks) * block_size >= (1ll << 31) ||
+      static_cast<long long>(max_suffix_blocks) * block_size >= (1ll << 31))
+    return pa::fail(PA_ERR_INVALID, "shared prefix: pool or table too large for 32-bit token indices");
+  if (partition_size < 0 ||
+      (partition_size > 0 && (partition_size % block_size != 0 || partition_size % pa::kChunkTokens != 0)))
+    return pa::fail(PA_ERR_INVALID, "shared prefix: partition_size must be 0 or a multiple of block_size and 16");
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return pa::fail(PA_ERR_INVALID, "shared prefix: scale must be finite");
+  if (num_seqs == 0) return pa::ok();
+  if (!q || !k_cache || !v_cache || !suffix_tables || !suffix_lens || !out || (prefix_len > 0 && !prefix_blocks))
+    return pa::fail(PA_ERR_INVALID, "shared prefix: null pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return pa::fail(PA_ERR_INVALID, "shared prefix: q, caches and out must be 16-byte aligned");
+  if (prefix_len == 0)
+    return pa_decode_attention(q, k_cache, v_cache, num_blocks, suffix_tables, max_suffix_blocks, suffix_lens,
+                               num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale, partition_size,
+                               workspace, workspace_bytes, out, dtype, stream);
+  const size_t need = pa_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, prefix_len, max_suffix_blocks,
+                                                      block_size, partition_size);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return pa::fail(PA_ERR_INVALID, "shared prefix: workspace missing, too small (need " + std::to_string(need) +
+                                        " bytes) or misaligned");
+  DecodeArgs a{q,        k_cache,      v_cache,     num_blocks, suffix_tables, max_suffix_blocks,
+               suffix_lens, num_seqs,  num_q_heads, num_kv_heads, head_dim,  block_size,
+               scale,    partition_size, workspace, out,          dtype,       static_cast<cudaStream_t>(stream)};
+  a.table_stride = suffix_table_stride;
+  a.part_offset = prefix_splits(prefix_len);
+  a.total_parts = a.part_offset + max_parts(max_suffix_blocks, block_size, partition_size);
+  const PrefixArgs pf{prefix_blocks, prefix_len};
+  pa_status st = dtype == PA_F16 ? dispatch_prefix<__half>(a, pf) : dispatch_prefix<__nv_bfloat16>(a, pf);
+  if (st != PA_OK) return st;
+  st = dtype == PA_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+  return st == PA_OK ? pa::ok() : st;
 }
 
 pa_status pa_device_error(int32_t* code_out, int32_t reset) {

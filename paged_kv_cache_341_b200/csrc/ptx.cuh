@@ -113,6 +113,13 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return pol;
 }
 
+// L2 policy for data many CTAs read again soon (a shared prefix).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // 3-D tile load global -> shared through a tensor map, completing on `bar`.
 // The innermost coordinate c0 is always 0 here (16-byte aligned).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,

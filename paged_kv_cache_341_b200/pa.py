@@ -47,6 +47,9 @@ SIGNATURES = {
                                    _vp, _sz, _vp, _i32, _vp]),
     "pa_decode_attention_static": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32,
                                           _i32, _vp, _i32, _vp]),
+    "pa_shared_prefix_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "pa_decode_attention_shared_prefix": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _vp, _i32, _i32,
+                                                 _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _i32, _vp]),
     "pa_device_error": (_i32, [_p32, _i32]),
     "pa_last_error": (ctypes.c_char_p, []),
 }
@@ -242,6 +245,43 @@ def pa_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale, 
                                     _dev(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, float(scale),
                                     int(partition_size), ws_ptr, ws_bytes, _dev(out, "out", k_cache.dtype), code,
                                     _stream(stream)))
+
+
+def pa_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, prefix_len, max_suffix_blocks, block_size,
+                                    partition_size):
+    return int(_lib.pa_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, prefix_len, max_suffix_blocks,
+                                                    block_size, partition_size))
+
+
+def pa_decode_attention_shared_prefix(q, k_cache, v_cache, prefix_blocks, prefix_len, suffix_tables, suffix_lens,
+                                      scale, out, partition_size=0, workspace=None, stream=None):
+    """Decode attention over a prefix shared by every sequence followed by each sequence's own suffix.
+
+    prefix_blocks: int32 CUDA [prefix_len / block_size]; suffix_tables: int32 CUDA [S, >= max suffix blocks]
+    (a row-slice view of a wider table is fine: its row stride is passed); suffix_lens: int32 CUDA [S].
+    The workspace (pa_shared_prefix_workspace_size bytes) is allocated here through torch when not given.
+    """
+    s, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != (s, hq, d):
+        raise ValueError("shape mismatch between q, caches and out")
+    if suffix_tables.dim() != 2 or suffix_tables.stride(1) != 1:
+        raise ValueError("suffix_tables must be a 2-D tensor with unit column stride")
+    if suffix_tables.dtype != torch.int32 or not suffix_tables.is_cuda:
+        raise TypeError("suffix_tables must be an int32 CUDA tensor")
+    max_suffix = suffix_tables.shape[1]
+    if workspace is None:
+        nbytes = pa_shared_prefix_workspace_size(s, hq, d, int(prefix_len), max_suffix, bs, int(partition_size))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    code = DTYPE_CODE[k_cache.dtype]
+    pb = _dev(prefix_blocks, "prefix_blocks", torch.int32) if int(prefix_len) > 0 else None
+    _check(_lib.pa_decode_attention_shared_prefix(
+        _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype), nb,
+        pb, int(prefix_len), ctypes.c_void_p(suffix_tables.data_ptr()), suffix_tables.stride(0), max_suffix,
+        _dev(suffix_lens, "suffix_lens", torch.int32), s, hq, hkv, d, bs, float(scale), int(partition_size),
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
+        _dev(out, "out", k_cache.dtype), code, _stream(stream)))
+    return workspace
 
 
 STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024

@@ -1,0 +1,111 @@
+"""GPU parity of the shared-prefix (cascade) decode against the oracle: the
+result must equal plain attention over prefix ++ suffix for every sequence.
+Tolerance as for every 16-bit cache: |gpu - ref| <= 2e-2 + 1e-2 |ref|."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle_decode
+from gpu_cases import TORCH, AsF64, assert_close, build_pool_contents
+from paged_kv_cache_341_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_cache_341_b200 import build
+    build.ensure_built()
+    from paged_kv_cache_341_b200 import pa as mod
+    assert mod.pa_device_error(reset=True) == 0
+    return mod
+
+
+def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed):
+    from paged_kv_cache_341_b200.cache import PagedKVCache
+    rng = np.random.default_rng(seed)
+    s = len(suffixes)
+    pblocks = prefix_len // bs
+    sblocks = [-(-n // bs) for n in suffixes]
+    nb = pblocks + sum(sblocks) + 4
+    mb = pblocks + max(sblocks + [1]) + 1
+    cache = PagedKVCache(nb, bs, hkv, d, TORCH[dtype], s, mb, initial_free_order=rng.permutation(nb))
+    if prefix_len:
+        cache.allocate(0, prefix_len)
+        for r in range(1, s):
+            cache.share(0, r)
+    for r, n in enumerate(suffixes):
+        if n:
+            cache.tables[r, pblocks:pblocks + sblocks[r]] = cache.pool.pa_pool_alloc(sblocks[r])
+        cache.lens[r] = prefix_len + n
+    k_host, v_host = build_pool_contents((nb, bs, hkv, d), dtype, cache.tables, cache.lens, bs, seed)
+    cache.k_cache.copy_(k_host)
+    cache.v_cache.copy_(v_host)
+    cache.upload_tables()
+    q_host = workloads.randn((s, hq, d), dtype, seed + 2)
+    q = q_host.cuda()
+    scale = 1.0 / math.sqrt(d)
+    out = torch.full((s, hq, d), float("nan"), dtype=TORCH[dtype], device="cuda")
+    prefix_ids = cache.d_tables[0, :pblocks].contiguous()
+    suffix_tables = cache.d_tables[:, pblocks:]
+    suffix_lens = cache.d_lens - prefix_len
+    pa.pa_decode_attention_shared_prefix(q, cache.k_cache, cache.v_cache, prefix_ids, prefix_len, suffix_tables,
+                                         suffix_lens, scale, out, partition_size=partition)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+    ref = oracle_decode(q_host.double().numpy(), AsF64(k_host), AsF64(v_host),
+                        [list(r) for r in cache.tables], [int(x) for x in cache.lens], scale)
+    plain = torch.empty_like(out)
+    ws = pa.decode_workspace(s, hq, d, mb, bs, partition)
+    cache.attend(q, plain, scale, partition, ws)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), ref, plain.float().cpu().numpy()
+
+
+SUFFIXES = [0, 1, 15, 16, 17, 100, 33]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (16, 4), (16, 2)])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("prefix_len", [32, 1088])
+@pytest.mark.parametrize("partition", [0, 64])
+def test_shared_prefix_matches_oracle(pa, dtype, d, hq, hkv, bs, prefix_len, partition):
+    gpu, ref, plain = run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, SUFFIXES, partition,
+                                  seed=prefix_len + bs + hq + d + partition)
+    tag = "dtype=%s d=%d hq=%d hkv=%d bs=%d prefix=%d p=%d" % (dtype, d, hq, hkv, bs, prefix_len, partition)
+    assert_close(gpu, ref, dtype, tag)
+    assert_close(gpu, plain.astype(np.float64), dtype, tag + " vs plain call")
+
+
+def test_many_sequences_and_row_tiles(pa):
+    rng = np.random.default_rng(5)
+    suffixes = [int(x) for x in rng.integers(0, 600, size=70)]
+    gpu, ref, _ = run_cascade(pa, "bf16", 32, 8, 128, 16, 2048 + 64, suffixes, 512, seed=6)
+    assert_close(gpu, ref, "bf16", "70 sequences")
+
+
+def test_zero_prefix_is_the_plain_call(pa):
+    gpu, ref, plain = run_cascade(pa, "bf16", 8, 2, 128, 16, 0, [5, 40], 0, seed=7)
+    assert_close(gpu, ref, "bf16", "no prefix")
+    assert np.array_equal(gpu, plain)
+
+
+def test_rejects_bad_arguments(pa):
+    q = torch.zeros(2, 8, 128, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(4, 16, 2, 128, dtype=torch.float32, device="cuda")
+    tables = torch.zeros(2, 2, dtype=torch.int32, device="cuda")
+    lens = torch.zeros(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(pa.PagedAttnError) as e:
+        pa.pa_decode_attention_shared_prefix(q, kc, kc, tables[0], 16, tables, lens, 0.1, q)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+    qb, kb = q.bfloat16(), kc.bfloat16()
+    with pytest.raises(pa.PagedAttnError) as e:
+        pa.pa_decode_attention_shared_prefix(qb, kb, kb, tables[0], 24, tables, lens, 0.1, qb)
+    assert e.value.status == pa.PA_ERR_INVALID
