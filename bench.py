@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_gqa")
     ap.add_argument("--partition", type=int, default=None, help="override the workload's partition size")
     ap.add_argument("--block-size", type=int, default=None, help="override the workload's block size")
+    ap.add_argument("--host-prefix-cache", action="store_true",
+                    help="time prompt allocation through the prefix cache on the host (no GPU)")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix workload: attend the shared prefix once for all sequences "
                          "(pa_decode_attention_shared_prefix)")
@@ -481,8 +483,47 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_host_prefix_cache(args):
+    """Host throughput of prompt allocation through the content-keyed prefix cache
+    (shared-prefix workload prompts: 200 x (30,720 shared + private suffix) tokens):
+    the library (C++) against the oracle (Python) on a bounded sample."""
+    from oracle import OraclePool
+    from paged_kv_cache_341_b200 import pa, workloads
+    w = workloads.get("shared_prefix")
+    lens = workloads.lengths(w)
+    rng = np.random.default_rng(w.seed)
+    system = [int(x) for x in rng.integers(0, 32000, size=w.shared_prefix)]
+    prompts = [system + [int(x) for x in rng.integers(0, 32000, size=int(n))] for n in lens]
+    tokens = sum(len(p) for p in prompts)
+    pool = pa.Pool(w.num_blocks, w.block_size)
+    pool.pa_pool_enable_prefix_cache()
+    table = np.full(w.max_blocks_per_seq, -1, np.int32)
+    arrays = [np.asarray(p, np.int32) for p in prompts]
+    t0 = time.perf_counter()
+    cached = 0
+    for a in arrays:
+        cached += pool.pa_seq_alloc_prompt(a, table)
+    lib_s = time.perf_counter() - t0
+    sample = prompts[:3]
+    op = OraclePool(w.num_blocks, w.block_size)
+    op.enable_prefix_cache()
+    t0 = time.perf_counter()
+    for p in sample:
+        op.alloc_prompt(p)
+    ora_s = time.perf_counter() - t0
+    line = {"metric": "prefix-cache prompt allocation, host tokens/s", "unit": "tokens/s",
+            "value": round(tokens / lib_s, 1), "prompts": len(prompts), "tokens": tokens,
+            "cached_tokens": cached, "blocks_used": w.num_blocks - pool.pa_pool_num_free(),
+            "oracle": {"value": round(sum(len(p) for p in sample) / ora_s, 1), "unit": "tokens/s",
+                       "sample": "first %d prompts" % len(sample)}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.host_prefix_cache:
+        run_host_prefix_cache(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -126,6 +126,33 @@ pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, in
                            int32_t num_seqs, int64_t* slots_out, int32_t* pairs_out,
                            int32_t* num_pairs_out);
 
+/* Prefix caching by block content ("Paged Attention", aidolsgroup.com, "Why
+ * it matters": every KV-cache block is hashed by its tokens and the tokens
+ * before it, so requests sharing a system prompt reuse the same blocks).
+ * Key of full block i of a prompt: 64-bit FNV-1a over the little-endian bytes
+ * of the int32 token ids tokens[0 : (i+1)*block_size].  Only full blocks are
+ * registered; a block leaves the cache when it returns to the free list. */
+pa_status pa_pool_enable_prefix_cache(pa_pool* pool);
+
+/* Blocks for a new sequence holding the prompt tokens[0..num_tokens): the
+ * leading full blocks whose key is registered (and whose stored token ids
+ * match) are shared (reference count + 1); the search stops at the first
+ * miss; the remaining blocks come from the front of the free list and each new
+ * full block is registered unless its key already is.  table[0 ..
+ * ceil(num_tokens/block_size)) receives the blocks; *num_cached_tokens the
+ * tokens whose K/V are already present (a multiple of block_size) -- the
+ * caller writes K/V for the rest.  All or nothing.  Errors: PA_ERR_EXHAUSTED,
+ * PA_ERR_INVALID (cache not enabled, table too small, bad argument). */
+pa_status pa_seq_alloc_prompt(pa_pool* pool, const int32_t* tokens, int32_t num_tokens, int32_t* table,
+                              int32_t table_cap, int32_t* num_cached_tokens);
+
+/* Number of blocks currently findable by key. */
+pa_status pa_pool_cached_blocks(const pa_pool* pool, int32_t* out);
+
+/* The key function itself: FNV-1a 64 of tokens[0..num_tokens) continued from
+ * `seed` (0 = the FNV offset basis). */
+pa_status pa_prefix_hash(const int32_t* tokens, int32_t num_tokens, uint64_t seed, uint64_t* out);
+
 /* ------------------------------------------------------------------------ */
 /* Device kernels (sm_100a).                                                */
 /* ------------------------------------------------------------------------ */

@@ -33,12 +33,12 @@ fp64) and the worked example printed on the agentechip page.  No function
 here is "parity unpinned".
 """
 
-from .pool import OraclePool, PoolExhausted, RefcountError, InvalidRequest
+from .pool import OraclePool, PoolExhausted, RefcountError, InvalidRequest, fnv1a64, token_bytes
 from .cache_ops import oracle_append, oracle_copy_blocks
 from .attention import gather_kv, oracle_decode, oracle_decode_one
 
 __all__ = [
-    "OraclePool", "PoolExhausted", "RefcountError", "InvalidRequest",
+    "OraclePool", "PoolExhausted", "RefcountError", "InvalidRequest", "fnv1a64", "token_bytes",
     "oracle_append", "oracle_copy_blocks",
     "gather_kv", "oracle_decode", "oracle_decode_one",
 ]

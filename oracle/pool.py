@@ -31,6 +31,26 @@ Plain Python lists on purpose: slow, but each rule above is one visible line.
 """
 
 
+FNV_OFFSET = 0xCBF29CE484222325
+FNV_PRIME = 0x100000001B3
+
+
+def fnv1a64(data, h=FNV_OFFSET):
+    """64-bit FNV-1a of a byte string, continued from ``h``."""
+    for byte in data:
+        h ^= byte
+        h = (h * FNV_PRIME) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def token_bytes(tokens):
+    """int32 token ids as little-endian bytes (the key's input)."""
+    out = bytearray()
+    for t in tokens:
+        out += (int(t) & 0xFFFFFFFF).to_bytes(4, "little")
+    return bytes(out)
+
+
 class PoolExhausted(RuntimeError):
     """No free block is left for a request (the pages' "KV cache exhausted")."""
 
@@ -57,6 +77,8 @@ class OraclePool:
                 raise InvalidRequest("initial_free_order must be a permutation of 0..N-1")
         self.free_list = order
         self.refcounts = [0] * self.num_blocks
+        self.prefix_cache = None          # key -> block id, once enabled
+        self.block_key = {}               # registered block id -> (key, its token ids)
 
     # -- pool-level operations ------------------------------------------------
 
@@ -93,6 +115,7 @@ class OraclePool:
         for b in ids:
             self.refcounts[b] -= 1
             if self.refcounts[b] == 0:
+                self._forget(b)
                 self.free_list.append(b)
 
     def fork(self, ids):
@@ -104,6 +127,60 @@ class OraclePool:
                 raise RefcountError("cannot share free block %d" % b)
         for b in ids:
             self.refcounts[b] += 1
+
+    # -- prefix caching by block content --------------------------------------
+    # "Paged Attention" (aidolsgroup.com), "Why it matters": a block is hashed
+    # by its tokens and the tokens before it, so prompts sharing a prefix share
+    # its blocks.  Key of full block i: FNV-1a 64 of the bytes of tokens
+    # [0, (i+1)*block_size).  Only full blocks are registered; the first block
+    # registered under a key keeps it; a block leaves the cache when freed.
+
+    def enable_prefix_cache(self):
+        if self.prefix_cache is None:
+            self.prefix_cache = {}
+
+    def _forget(self, b):
+        if self.prefix_cache is None or b not in self.block_key:
+            return
+        key, _ = self.block_key.pop(b)
+        if self.prefix_cache.get(key) == b:
+            del self.prefix_cache[key]
+
+    def alloc_prompt(self, tokens):
+        """Table (list of block ids) for a new sequence holding ``tokens``, and
+        how many leading tokens sit in blocks found in the cache."""
+        if self.prefix_cache is None:
+            raise InvalidRequest("prefix cache not enabled")
+        bs = self.block_size
+        n = len(tokens)
+        nblocks = -(-n // bs)
+        keys = []
+        h = FNV_OFFSET
+        for i in range(n // bs):
+            # FNV-1a is a byte stream: continuing it over block i's bytes gives the
+            # hash of everything up to the end of block i
+            h = fnv1a64(token_bytes(tokens[i * bs:(i + 1) * bs]), h)
+            keys.append(h)
+        table = []
+        for i, key in enumerate(keys):
+            b = self.prefix_cache.get(key)
+            if b is None or self.block_key[b][1] != list(tokens[i * bs:(i + 1) * bs]):
+                break
+            table.append(b)
+        hits = len(table)
+        if nblocks - hits > len(self.free_list):
+            raise PoolExhausted("KV cache exhausted: %d blocks requested, %d free" % (nblocks - hits,
+                                                                                      len(self.free_list)))
+        for b in table:
+            self.refcounts[b] += 1
+        for i in range(hits, nblocks):
+            b = self.free_list.pop(0)
+            self.refcounts[b] = 1
+            table.append(b)
+            if i < len(keys) and keys[i] not in self.prefix_cache:
+                self.prefix_cache[keys[i]] = b
+                self.block_key[b] = (keys[i], list(tokens[i * bs:(i + 1) * bs]))
+        return table, hits * bs
 
     def refcount(self, b):
         self._check_id(b)

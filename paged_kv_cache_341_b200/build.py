@@ -23,7 +23,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v"]
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall"]
 SOURCES_CU = ["pa_device.cu"]
-SOURCES_CPP = ["pool.cpp", "common.cpp"]
+SOURCES_CPP = ["pool.cpp", "prefix_cache.cpp", "common.cpp"]
 
 
 def nvcc():

@@ -19,34 +19,7 @@
 #include "pa.h"
 #include "pa_common.h"
 
-struct pa_pool {
-  int32_t num_blocks = 0;
-  int32_t block_size = 0;
-  std::vector<int32_t> ring;      // free list storage, capacity num_blocks
-  int32_t head = 0;               // index of the front entry
-  int32_t count = 0;              // entries queued
-  std::vector<int32_t> refcount;  // per block id
-
-  int32_t pop_front() {
-    int32_t b = ring[head];
-    head = (head + 1 == num_blocks) ? 0 : head + 1;
-    --count;
-    return b;
-  }
-  void push_back(int32_t b) {
-    int32_t tail = head + count;
-    if (tail >= num_blocks) tail -= num_blocks;
-    ring[tail] = b;
-    ++count;
-  }
-  // Undo the most recent pop_front (used to roll back multi-step calls).
-  void unpop_front(int32_t b) {
-    head = (head == 0) ? num_blocks - 1 : head - 1;
-    ring[head] = b;
-    ++count;
-  }
-  bool valid_id(int32_t b) const { return b >= 0 && b < num_blocks; }
-};
+#include "pool_internal.h"
 
 extern "C" {
 
@@ -111,7 +84,10 @@ pa_status pa_pool_free(pa_pool* pool, const int32_t* ids, int32_t n) {
                                              " released more often than referenced");
   }
   for (int32_t i = 0; i < n; ++i)
-    if (--pool->refcount[ids[i]] == 0) pool->push_back(ids[i]);
+    if (--pool->refcount[ids[i]] == 0) {
+      pool->forget_hash(ids[i]);
+      pool->push_back(ids[i]);
+    }
   return pa::ok();
 }
 

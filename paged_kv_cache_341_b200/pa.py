@@ -40,6 +40,10 @@ SIGNATURES = {
     "pa_pool_export": (_i32, [_vp, _p32, _p32, _p32]),
     "pa_seq_reserve_slot": (_i32, [_vp, _p32, _i32, _p32, _p64, _p32, _p32]),
     "pa_reserve_slots": (_i32, [_vp, _p32, _i32, _p32, _i32, _p64, _p32, _p32]),
+    "pa_pool_enable_prefix_cache": (_i32, [_vp]),
+    "pa_seq_alloc_prompt": (_i32, [_vp, _p32, _i32, _p32, _i32, _p32]),
+    "pa_pool_cached_blocks": (_i32, [_vp, _p32]),
+    "pa_prefix_hash": (_i32, [_p32, _i32, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]),
     "pa_append_kv": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
@@ -191,6 +195,34 @@ class Pool:
                                      lens.ctypes.data_as(_p32), s, slots.ctypes.data_as(_p64),
                                      pairs.ctypes.data_as(_p32), ctypes.byref(npairs)))
         return slots, pairs[: npairs.value].copy()
+
+
+    # -- prefix caching ------------------------------------------------------
+
+    def pa_pool_enable_prefix_cache(self):
+        _check(_lib.pa_pool_enable_prefix_cache(self._h))
+
+    def pa_seq_alloc_prompt(self, tokens, table):
+        """Blocks for a prompt (``table``: writable int32 array); returns the number of cached tokens."""
+        arr, ptr = _i32_array(tokens)
+        if table.dtype != np.int32 or not table.flags.c_contiguous:
+            raise TypeError("table must be a contiguous int32 array")
+        cached = ctypes.c_int32()
+        _check(_lib.pa_seq_alloc_prompt(self._h, ptr, arr.size, table.ctypes.data_as(_p32), table.size,
+                                        ctypes.byref(cached)))
+        return cached.value
+
+    def pa_pool_cached_blocks(self):
+        out = ctypes.c_int32()
+        _check(_lib.pa_pool_cached_blocks(self._h, ctypes.byref(out)))
+        return out.value
+
+
+def pa_prefix_hash(tokens, seed=0):
+    arr, ptr = _i32_array(tokens)
+    out = ctypes.c_uint64()
+    _check(_lib.pa_prefix_hash(ptr, arr.size, seed, ctypes.byref(out)))
+    return out.value
 
 
 # --------------------------------------------------------------------------
