@@ -317,7 +317,8 @@ def run_ours(args):
     ws = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
     kv_bytes = sc.kv_bytes()
     config = workload_config(sc, args)
-    launches_per_step = (1 if pairs.shape[0] else 0) + 1 + (2 if part > 0 else 1)
+    # copy (when pairs) + append + planner + decode (+ merge with partitions)
+    launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 1 + 1 + (1 if part > 0 else 0)
     cascade = args.cascade and w.shared_prefix > 0
     if cascade:
         pblocks = w.shared_prefix // w.block_size
@@ -327,7 +328,7 @@ def run_ours(args):
         ws = torch.empty(pa.pa_shared_prefix_workspace_size(sc.batch, w.num_q_heads, w.head_dim, w.shared_prefix,
                                                             suffix_tables.shape[1], w.block_size, part),
                          dtype=torch.uint8, device="cuda")
-        launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 3
+        launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 4   # + prefix, planner, decode, merge
         config["cascade"] = {"prefix_tokens": w.shared_prefix, "unique_kv_bytes": sc.unique_kv_bytes()}
 
     def attend():

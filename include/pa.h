@@ -178,10 +178,11 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
                          int32_t head_dim, pa_dtype dtype, void* stream);
 
 /* Bytes of device workspace pa_decode_attention takes for these sizes: 256
- * bytes for the work-unit counter, plus, when partition_size > 0, one float32
- * partial (max, sum, D values) per (sequence, query head, partition), with
- * partitions = ceil(max_blocks_per_seq * block_size / partition_size).  0 for
- * invalid sizes. */
+ * bytes for the work-unit counter, a planned work-unit list of 16 bytes per
+ * (sequence, query head, partition) rounded up to 256 bytes, plus, when
+ * partition_size > 0, one float32 partial (max, sum, D values) per (sequence,
+ * query head, partition); partitions = ceil(max_blocks_per_seq * block_size /
+ * partition_size), or 1 when partition_size == 0.  0 for invalid sizes. */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_blocks_per_seq, int32_t block_size,
                                 int32_t partition_size);
@@ -211,9 +212,9 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
  *                  as a programmatic dependent of the first).
  *   workspace      device buffer of pa_decode_workspace_size() bytes, owned
  *                  by the caller; required when partition_size > 0.  With a
- *                  workspace the work units are handed out through a counter
- *                  in it; the counter is zeroed
- *                  by a cudaMemsetAsync on `stream` before each launch.  With
+ *                  workspace, a one-CTA planning kernel first lists the work
+ *                  units in it (full partitions, then the rest longest first)
+ *                  and the decode kernel takes them through a counter; with
  *                  NULL (only when partition_size == 0) the units are dealt
  *                  round-robin.  Calls sharing a workspace must not
  *                  overlap on the GPU.
@@ -229,8 +230,9 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
                               void* out, pa_dtype dtype, void* stream);
 
 /* Bytes of device workspace pa_decode_attention_shared_prefix takes: 256
- * bytes for the work-unit counter plus one float32 partial (max, sum, D
- * values) per (sequence, query head, part), where the parts are the prefix's
+ * bytes for the work-unit counter, the suffix's work-unit list (as for
+ * pa_decode_workspace_size) and one float32 partial (max, sum, D values) per
+ * (sequence, query head, part), where the parts are the prefix's
  * ceil(prefix_len / 1024) slices followed by the suffix's partitions
  * (ceil(max_suffix_blocks * block_size / partition_size), or 1 when
  * partition_size == 0).  0 for invalid sizes. */

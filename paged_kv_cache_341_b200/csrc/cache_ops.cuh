@@ -21,6 +21,7 @@ namespace pa {
 __global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                                                      const int64_t* __restrict__ slots, uint4* k_cache,
                                                      uint4* v_cache, int64_t num_slots, int row_vecs) {
+  allow_dependent_launch();   // a following planner reads only the lengths: it may start now
   const int t = blockIdx.x;
   const int64_t slot = slots[t];
   if (slot < 0) return;

@@ -10,11 +10,14 @@
 // Design (HBM-bound: every K/V byte is read exactly once):
 //
 // * Work unit = (sequence, partition of `partition_size` tokens, tile of HT
-//   KV heads).  Units are numbered in two passes over the sequences -- first
-//   every full partition, then every sequence's shorter remainder partition --
-//   and a persistent grid (one CTA per SM) takes them from an atomic counter
-//   in that order, so the small units come last and the SMs finish together.
-//   Without a workspace the units are dealt round-robin instead.
+//   KV heads).  plan_kernel lists the units -- every full partition in
+//   sequence order, then every remainder partition (or, without partitions,
+//   every whole sequence) longest first -- and the persistent grid takes them
+//   from an atomic counter in that order, so the small units come last and
+//   the SMs finish together.  The decode kernel is a programmatic dependent of
+//   the planner: its CTAs start while the plan is written and wait for it.
+//   Without a workspace the units are walked from the lengths and dealt
+//   round-robin instead.
 // * One producer warp streams each unit as chunks of 16 tokens, each chunk
 //   taken straight from the physical block the block table names, by TMA tile
 //   loads into a ring of shared-memory stages guarded by full/empty mbarriers.
@@ -70,7 +73,8 @@ struct DecodeParams {
   void* out;                     // [S][Hq][D]
   float* part_acc;               // [S][Hq][NP][D]   (partitioned mode)
   float2* part_ml;               // [S][Hq][NP]      (m in base-2 units, l)
-  int* sched;                    // unit counter (zeroed before launch), or null: static order
+  int* sched;                    // [0]: unit counter, [1]: number of planned units (plan_kernel)
+  const int4* units;             // planned unit list {seq, part, tile, len}, or null: walk the sequences
   int table_stride;              // elements between rows of block_tables (>= max_blocks)
   int part_offset;               // partial index of partition 0 (shared-prefix mode)
   int force_partials;            // write partials even for single-partition sequences
@@ -206,7 +210,7 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
     }
     win_total = __shfl_sync(0xffffffffu, my_incl, 31);
   };
-  load_window();
+  if (prm.units == nullptr) load_window();
 
   int stage = 0;
   uint32_t phase = 0;
@@ -216,50 +220,69 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
   int tw_seq = -1, tw_base = -1, tw_val = 0;
   bool ok = true;
 
-  // Next unit index: from the shared counter, claimed one unit ahead by lane
-  // 0 so the atomic's round trip overlaps the current unit; round-robin when
-  // there is no counter.
-  int claimed = 0;
-  if (prm.sched && lane == 0) claimed = atomicAdd(prm.sched, 1);
+  // Planned order: claim the next unit index and fetch its descriptor one
+  // unit ahead (lane 0), so both round trips overlap the current unit.
+  const bool planned = prm.units != nullptr;
+  int total_units = 0;
+  int4 next_desc = make_int4(-1, 0, 0, 0);
+  auto claim = [&]() {
+    int4 d = make_int4(-1, 0, 0, 0);
+    if (lane == 0) {
+      const int c = atomicAdd(prm.sched, 1);
+      if (c < total_units) d = __ldcg(prm.units + c);
+    }
+    return d;
+  };
+  if (planned) {
+    wait_prerequisite_grids();                       // the plan is complete and visible
+    if (lane == 0) total_units = __ldcg(prm.sched + 1);
+    total_units = __shfl_sync(0xffffffffu, total_units, 0);
+    next_desc = claim();
+  }
   int rr = blockIdx.x;
 
   while (ok) {
-    int u;
-    if (prm.sched) {
-      u = __shfl_sync(0xffffffffu, claimed, 0);
+    int seq, len, part, tile;
+    if (planned) {
+      const int4 d = make_int4(__shfl_sync(0xffffffffu, next_desc.x, 0), __shfl_sync(0xffffffffu, next_desc.y, 0),
+                               __shfl_sync(0xffffffffu, next_desc.z, 0), __shfl_sync(0xffffffffu, next_desc.w, 0));
+      if (d.x < 0) break;
+      next_desc = claim();
+      seq = d.x;
+      part = d.y;
+      tile = d.z;
+      len = d.w;
     } else {
-      u = rr;
+      const int u = rr;
       rr += gridDim.x;
-    }
-    bool exhausted = false;
-    while (u >= win_base + win_total) {
-      win_base += win_total;
-      win_s0 += 32;
-      if (win_s0 >= S) {
-        if (pass == 1) {
-          exhausted = true;
-          break;
+      bool exhausted = false;
+      while (u >= win_base + win_total) {
+        win_base += win_total;
+        win_s0 += 32;
+        if (win_s0 >= S) {
+          if (pass == 1) {
+            exhausted = true;
+            break;
+          }
+          pass = 1;
+          win_s0 = 0;
         }
-        pass = 1;
-        win_s0 = 0;
+        load_window();
       }
-      load_window();
-    }
-    if (exhausted) break;
-    if (prm.sched && lane == 0) claimed = atomicAdd(prm.sched, 1);
-    const unsigned hit = __ballot_sync(0xffffffffu, win_base + my_incl > u);
-    const int hl = __ffs(hit) - 1;
-    const int seq = win_s0 + hl;
-    const int len = __shfl_sync(0xffffffffu, my_len, hl);
-    const int excl = __shfl_sync(0xffffffffu, my_incl - my_units, hl);
-    const int r = u - (win_base + excl);
-    int part, tile;
-    if (pass == 0) {
-      part = r / n_tiles;
-      tile = r - part * n_tiles;
-    } else {
-      part = len / P;
-      tile = r;
+      if (exhausted) break;
+      const unsigned hit = __ballot_sync(0xffffffffu, win_base + my_incl > u);
+      const int hl = __ffs(hit) - 1;
+      seq = win_s0 + hl;
+      len = __shfl_sync(0xffffffffu, my_len, hl);
+      const int excl = __shfl_sync(0xffffffffu, my_incl - my_units, hl);
+      const int r = u - (win_base + excl);
+      if (pass == 0) {
+        part = r / n_tiles;
+        tile = r - part * n_tiles;
+      } else {
+        part = len / P;
+        tile = r;
+      }
     }
     const int nparts = parts_of(len, P);
     const int tok_begin = P > 0 ? part * P : 0;
@@ -668,8 +691,10 @@ __device__ __forceinline__ uint32_t swz(int tok, int chunk) {
   return static_cast<uint32_t>(tok * kSwizzleBytes + ((chunk ^ (tok & 7)) << 4));
 }
 
+// 128 registers: eight 64-thread CTAs (the default launch shape) fill the
+// register file exactly.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
+__global__ void __maxnreg__(128)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeParams prm) {
   static_assert(sizeof(T) == 2, "tensor-core consumer takes 16-bit caches");
@@ -874,6 +899,134 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
       ++units_done;
     }
   }
+}
+
+// ===========================================================================
+// Planner: the decode kernel's unit list.  Full partitions first, in
+// sequence order with the KV-head tiles of a partition next to each other
+// (they read the same blocks); then the remainder partitions -- or, without
+// partitions, the whole sequences -- by decreasing length (counting sort on
+// 16-token chunks), so the smallest units are taken last.  One CTA; also
+// zeroes the unit counter and stores the unit count.  It is launched as a
+// programmatic dependent of the kernel before it (the append of the step) and
+// reads only the lengths, so it overlaps that kernel; before exiting it waits
+// for it, so a decode grid that has waited for the planner also sees the
+// appended K/V.
+// ===========================================================================
+struct PlanParams {
+  const int32_t* context_lens;
+  int4* units;                   // {seq, part, tile, len}
+  int* header;                   // [0] unit counter (zeroed), [1] unit count
+  int num_seqs, partition_size, num_tiles, cap;
+};
+
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 4096;     // remainder sizes in 16-token chunks; longer ones share the last
+
+// Exclusive prefix sum over the CTA; *total receives the sum.  All threads call it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += t;
+    }
+    if (lane < nw) warp_sums[lane] = w;       // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = warp > 0 ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before + incl - v;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm) {
+  __shared__ int bucket[kPlanBuckets];
+  __shared__ int warp_sums[32];
+  allow_dependent_launch();                    // the decode grid may start; it waits for this one
+  const int tid = threadIdx.x;
+  const int S = prm.num_seqs, P = prm.partition_size, nt = prm.num_tiles;
+  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) bucket[b] = 0;
+  __syncthreads();
+  auto load_len = [&](int s) {
+    int len = prm.context_lens[s];
+    return len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
+  };
+  auto rem_bucket = [&](int len) {               // -1: no remainder unit
+    int rem;
+    if (P > 0) {
+      if (len % P == 0 && len > 0) return -1;
+      rem = len % P;
+    } else {
+      rem = len;
+    }
+    const int chunks = (rem + kChunkTokens - 1) / kChunkTokens;
+    return chunks < kPlanBuckets ? chunks : kPlanBuckets - 1;
+  };
+  // pass 0: full partitions, and the remainder histogram
+  int written = 0;
+  for (int base = 0; base < S; base += kPlanThreads) {
+    const int s = base + tid;
+    int len = 0, nfull = 0;
+    if (s < S) {
+      len = load_len(s);
+      nfull = P > 0 ? len / P : 0;
+      const int b = rem_bucket(len);
+      if (b >= 0) atomicAdd(&bucket[b], 1);
+    }
+    int round_total;
+    const int off = block_exclusive_scan(nfull * nt, warp_sums, &round_total);
+    for (int p = 0; p < nfull; ++p)
+      for (int t = 0; t < nt; ++t) prm.units[written + off + p * nt + t] = make_int4(s, p, t, len);
+    written += round_total;
+  }
+  // bucket starts, largest remainders first: start[b] = written + nt * sum_{b' > b} count[b']
+  {
+    constexpr int PER = kPlanBuckets / kPlanThreads;
+    int local[PER];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      local[i] = bucket[kPlanBuckets - 1 - (tid * PER + i)];   // reversed order
+      sum += local[i];
+    }
+    int tot;
+    const int off = block_exclusive_scan(sum, warp_sums, &tot);
+    int run = off;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int b = kPlanBuckets - 1 - (tid * PER + i);
+      const int c = local[i];
+      bucket[b] = written + run * nt;             // becomes the cursor of bucket b
+      run += c;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      prm.header[0] = 0;
+      prm.header[1] = written + tot * nt;
+    }
+  }
+  // pass 1: remainder partitions into their buckets
+  for (int s = tid; s < S; s += kPlanThreads) {
+    const int len = load_len(s);
+    const int b = rem_bucket(len);
+    if (b < 0) continue;
+    const int pos = atomicAdd(&bucket[b], nt);
+    const int part = P > 0 ? len / P : 0;
+    for (int t = 0; t < nt; ++t) prm.units[pos + t] = make_int4(s, part, t, len);
+  }
+  wait_prerequisite_grids();
 }
 
 // ===========================================================================

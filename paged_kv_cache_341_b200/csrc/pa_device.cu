@@ -92,7 +92,14 @@ struct DecodeArgs {
   int total_parts = 0;           // 0: ceil(max_blocks*block_size/P), else the partial row stride
 };
 
-constexpr size_t kSchedBytes = 256;   // unit counter at the head of the workspace
+constexpr size_t kSchedBytes = 256;   // unit counter and unit count at the head of the workspace
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Planned unit list: at most S * n_tiles * parts units (n_tiles <= Hkv <= Hq).
+size_t units_bytes(long long S, long long Hq, long long parts) {
+  return round256(static_cast<size_t>(S) * Hq * parts * sizeof(int4));
+}
 
 int max_parts(int max_blocks, int block_size, int P) {
   if (P <= 0) return 1;
@@ -211,11 +218,13 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.block_tables = a.block_tables;
   prm.context_lens = a.context_lens;
   prm.out = a.out;
-  // workspace: [unit counter, 256 B][partial outputs][partial (m, l)]
+  // workspace: [unit counter + count, 256 B][unit list][partial outputs][partial (m, l)]
   const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
   char* ws = static_cast<char*>(a.workspace);
+  const size_t list_bytes = units_bytes(a.S, a.Hq, max_parts(a.max_blocks, a.BS, a.P));
   prm.sched = ws ? reinterpret_cast<int*>(ws) : nullptr;
-  prm.part_acc = partials ? reinterpret_cast<float*>(ws + kSchedBytes) : nullptr;
+  prm.units = ws ? reinterpret_cast<const int4*>(ws + kSchedBytes) : nullptr;
+  prm.part_acc = partials ? reinterpret_cast<float*>(ws + kSchedBytes + list_bytes) : nullptr;
   prm.part_ml = partials ? reinterpret_cast<float2*>(prm.part_acc + acc_elems) : nullptr;
   prm.table_stride = a.table_stride > 0 ? a.table_stride : a.max_blocks;
   prm.part_offset = a.part_offset;
@@ -235,13 +244,42 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.q_bytes = static_cast<uint32_t>(q_bytes);
   prm.qk_scale = a.scale * 1.4426950408889634f;
 
-  if (prm.sched) {
-    // the unit counter starts at zero on every launch
-    e = cudaMemsetAsync(prm.sched, 0, sizeof(int), a.stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(unit counter)");
+  if (prm.units) {
+    // planner (one CTA), then the decode grid as its programmatic dependent
+    pa::PlanParams pp;
+    pp.context_lens = a.context_lens;
+    pp.units = reinterpret_cast<int4*>(ws + kSchedBytes);
+    pp.header = prm.sched;
+    pp.num_seqs = a.S;
+    pp.partition_size = a.P;
+    pp.num_tiles = n_tiles;
+    pp.cap = a.max_blocks * a.BS;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pcfg = {};
+    pcfg.gridDim = dim3(1);
+    pcfg.blockDim = dim3(pa::kPlanThreads);
+    pcfg.stream = a.stream;
+    pcfg.attrs = pdl;
+    pcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pcfg, pa::plan_kernel, pp);
+    if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, prm);
+  } else {
+    kern<<<grid, threads, smem, a.stream>>>(tm_k, tm_v, prm);
+    e = cudaGetLastError();
   }
-  kern<<<grid, threads, smem, a.stream>>>(tm_k, tm_v, prm);
-  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_kernel launch");
 
   if (partials) {
@@ -333,10 +371,11 @@ pa_status launch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   const int np = a.total_parts;
   const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
   char* ws = static_cast<char*>(a.workspace);
+  const size_t list_bytes = units_bytes(a.S, a.Hq, max_parts(a.max_blocks, a.BS, a.P));
   pa::PrefixParams prm;
   prm.q = a.q;
   prm.prefix_blocks = pf.prefix_blocks;
-  prm.part_acc = reinterpret_cast<float*>(ws + kSchedBytes);
+  prm.part_acc = reinterpret_cast<float*>(ws + kSchedBytes + list_bytes);
   prm.part_ml = reinterpret_cast<float2*>(prm.part_acc + acc_elems);
   prm.num_seqs = a.S;
   prm.num_q_heads = a.Hq;
@@ -429,9 +468,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
   if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||
       partition_size < 0)
     return 0;
-  if (partition_size == 0) return kSchedBytes;
   const size_t np = static_cast<size_t>(max_parts(max_blocks_per_seq, block_size, partition_size));
-  return kSchedBytes + static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
+  const size_t list = units_bytes(num_seqs, num_q_heads, np);
+  if (partition_size == 0) return kSchedBytes + list;
+  return kSchedBytes + list + static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
 }
 
 pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_cache, int32_t num_blocks,
@@ -538,9 +578,10 @@ size_t pa_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
   if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || prefix_len < 0 || max_suffix_blocks <= 0 ||
       block_size <= 0 || partition_size < 0)
     return 0;
-  const size_t np = static_cast<size_t>(prefix_splits(prefix_len)) +
-                    static_cast<size_t>(max_parts(max_suffix_blocks, block_size, partition_size));
-  return kSchedBytes + static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
+  const size_t suffix_parts = static_cast<size_t>(max_parts(max_suffix_blocks, block_size, partition_size));
+  const size_t np = static_cast<size_t>(prefix_splits(prefix_len)) + suffix_parts;
+  return kSchedBytes + units_bytes(num_seqs, num_q_heads, suffix_parts) +
+         static_cast<size_t>(num_seqs) * num_q_heads * np * (static_cast<size_t>(head_dim) * 4 + 8);
 }
 
 pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, const void* v_cache,

@@ -70,8 +70,10 @@ class Workload:
 
 WORKLOADS = {
     "tiny_fp32": Workload("tiny_fp32", 1, 4, 2, 2, 64, 16, "f32"),
-    "llama2_7b_mha": Workload("llama2_7b_mha", 2, 64, 32, 32, 128, 16, "f16", partition_size=512),
-    "llama3_8b_gqa": Workload("llama3_8b_gqa", 3, 256, 32, 8, 128, 16, "bf16", partition_size=512),
+    # partition sizes: the 70B-shaped workload states 512; for the Llama shapes, which state
+    # none, 1,024 was the fastest of 256/512/1,024/2,048 on B200
+    "llama2_7b_mha": Workload("llama2_7b_mha", 2, 64, 32, 32, 128, 16, "f16", partition_size=1024),
+    "llama3_8b_gqa": Workload("llama3_8b_gqa", 3, 256, 32, 8, 128, 16, "bf16", partition_size=1024),
     "shared_prefix": Workload("shared_prefix", 4, 200, 32, 8, 128, 16, "bf16", partition_size=512,
                               shared_prefix=30720),
     "long_70b_gqa": Workload("long_70b_gqa", 5, 8, 64, 8, 128, 32, "bf16", partition_size=512),

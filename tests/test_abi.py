@@ -66,9 +66,11 @@ def test_decode_rejects_bad_arguments_on_host(built_library):
 
 def test_workspace_size_formula(built_library):
     from paged_kv_cache_341_b200 import pa
-    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 0) == 256
+    def units(parts):
+        return -(-8 * 64 * parts * 16 // 256) * 256
+    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 0) == 256 + units(1)
     np_ = -(-1026 * 32 // 512)
-    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 512) == 256 + 8 * 64 * np_ * (128 * 4 + 8)
+    assert pa.pa_decode_workspace_size(8, 64, 128, 1026, 32, 512) == 256 + units(np_) + 8 * 64 * np_ * (128 * 4 + 8)
     assert pa.pa_decode_workspace_size(0, 64, 128, 1026, 32, 512) == 0
 
 
