@@ -4,16 +4,17 @@ One step = one decode step of one attention layer over the whole batch of the
 Llama-3-8B-shaped GQA workload (256 sequences, 32 query / 8 KV heads,
 head_dim 128, block 16, bf16 cache, log-normal lengths with median 1024
 clipped to [16, 8192]): copy-on-write copies, append of one new token per
-sequence, and split-context attention (512-token partitions + merge).
+sequence, and split-context attention (1,024-token partitions + merge).
 
 ``value``: KV GB/s = algorithmic K/V bytes of a step (every (token, KV head)
 row of K and V once) / device time of a step, inputs resident in HBM, the same
 decode step repeated (appends rewrite the same slots, so the workload stays
-the stated one).  The K/V set (1.7 GB) is far larger than L2 (126 MB), so no
+the stated one).  The K/V set (1.88 GB) is far larger than L2 (126 MB), so no
 flush is needed between steps.  ``e2e``: the same metric through the public
 API from pinned host buffers: every step reserves its slots on the host,
-copies q / new K,V / slots / tables to the device, runs the kernels and reads
-the output back (sequences grow by one token per step there).
+copies q / new K,V and one metadata block (slots, lengths, changed table
+entries, copy pairs) to the device, runs the kernels and reads the output back
+(sequences grow by one token per step there).
 
 ``--impl reference`` times the CPU oracle (float64 numpy) on a bounded sample
 of the same workload.  Under torchrun every rank runs its own replica of the
@@ -52,7 +53,7 @@ def parse():
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix workload: attend the shared prefix once for all sequences "
                          "(pa_decode_attention_shared_prefix)")
-    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=120)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -390,7 +391,9 @@ def run_ours(args):
         for i in range(n_e2e):
             qi, ki, vi = sc.step_inputs(1 + i)
             host_in.append((qi.pin_memory(), ki.pin_memory(), vi.pin_memory()))
-        copy_stream = torch.cuda.Stream()
+        # H2D and D2H on streams of their own (separate copy engines): step i+1's
+        # inputs travel while step i computes, step i's output while step i+1 does
+        h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
         dev_in = [(torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)) for _ in range(2)]
         dev_out = [torch.empty_like(out) for _ in range(2)]
         host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
@@ -398,7 +401,7 @@ def run_ours(args):
         comp_done = [torch.cuda.Event() for _ in range(2)]
         out_read = [torch.cuda.Event() for _ in range(2)]
         in_bytes = q.numel() * q.element_size() + 2 * kn.numel() * kn.element_size()
-        meta_bytes = (c.d_tables[sc.rows].numel() + c.d_lens[sc.rows].numel()) * 4 + sc.batch * 8
+        meta_bytes = c.step_metadata_bytes
         ws_e2e = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
         e2e_bytes, pairs_total = 0, 0
         if world > 1:
@@ -406,41 +409,47 @@ def run_ours(args):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        copy_stream.wait_stream(stream)
+        h2d_stream.wait_stream(stream)
+        d2h_stream.wait_stream(stream)
+        t_host = time.perf_counter()
         for i in range(n_e2e):
             b = i % 2
             qd, kd, vd = dev_in[b]
-            with torch.cuda.stream(copy_stream):
+            with torch.cuda.stream(h2d_stream):
                 if i >= 2:
-                    copy_stream.wait_event(comp_done[b])
+                    h2d_stream.wait_event(comp_done[b])     # step i-2 no longer reads these inputs
                 qi, ki, vi = host_in[i]
                 qd.copy_(qi, non_blocking=True)
                 kd.copy_(ki, non_blocking=True)
                 vd.copy_(vi, non_blocking=True)
-                in_ready[b].record(copy_stream)
+                in_ready[b].record(h2d_stream)
             stream.wait_event(in_ready[b])
             if i >= 2:
-                stream.wait_event(out_read[b])
+                stream.wait_event(out_read[b])              # step i-2's output has left dev_out[b]
             _, pr = c.decode_step(qd, kd, vd, dev_out[b], w.scale, part, ws_e2e, rows=sc.rows, stream=stream)
             pairs_total += pr.shape[0]
             e2e_bytes += sc.kv_bytes()
             comp_done[b].record(stream)
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(comp_done[b])
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(comp_done[b])
                 host_out[b].copy_(dev_out[b], non_blocking=True)
-                out_read[b].record(copy_stream)
-        stream.wait_stream(copy_stream)
+                out_read[b].record(d2h_stream)
+        t_host = time.perf_counter() - t_host
+        stream.wait_stream(h2d_stream)
+        stream.wait_stream(d2h_stream)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
         e2e_ms = max_over_ranks([e2e_ms], device="cuda")[0]
         e2e = {"value": round(whole_job_gbs(e2e_bytes, e2e_ms, world), 2), "unit": "GB/s",
-               "h2d_bytes_per_step": int(in_bytes + meta_bytes + 8 * pairs_total / max(1, n_e2e)),
+               "h2d_bytes_per_step": int(in_bytes + meta_bytes),
                "d2h_bytes_per_step": int(out.numel() * out.element_size()), "steps": n_e2e,
                "ms_per_step": round(e2e_ms / n_e2e, 4),
-               "note": "per step: host slot reservation, pinned H2D of q/new K,V/slots/tables, kernels, "
-                       "D2H of out; copies overlap the previous step's kernels; sequences grow one token "
-                       "per step"}
+               "copy_pairs_per_step": round(pairs_total / max(1, n_e2e), 2),
+               "host_issue_ms_per_step": round(1e3 * t_host / n_e2e, 4),
+               "note": "per step: host slot reservation, pinned H2D of q/new K,V and of one metadata "
+                       "block (slots, lengths, changed table entries, copy pairs), kernels, D2H of out; "
+                       "copies overlap the previous step's kernels; sequences grow one token per step"}
         assert pa.pa_device_error() == 0
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N=1 only)

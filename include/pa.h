@@ -177,6 +177,17 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
                          int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
                          int32_t head_dim, pa_dtype dtype, void* stream);
 
+/* Write changed block-table entries on the device: updates is a device int32
+ * [num_updates][3] array of (row, column, block id), applied to
+ * block_tables (device int32 [num_rows][table_stride]).  A host reservation
+ * changes at most one entry per appending sequence (a fresh block at a block
+ * boundary, or the private copy of a shared block), so sending the changes
+ * instead of the tables keeps a step's host-to-device traffic small.
+ * Out-of-range rows or columns are skipped and set the device error word (3).
+ * Entries with the same (row, column) in one call must not repeat. */
+pa_status pa_update_block_tables(int32_t* block_tables, int32_t num_rows, int32_t table_stride,
+                                 const int32_t* updates, int32_t num_updates, void* stream);
+
 /* Bytes of device workspace pa_decode_attention takes for these sizes: 256
  * bytes for the work-unit counter, a planned work-unit list of 16 bytes per
  * (sequence, query head, partition) rounded up to 256 bytes, plus, when

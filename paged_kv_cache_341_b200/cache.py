@@ -13,8 +13,10 @@ is one pass of the hot path through the C ABI:
    ``pa_decode_attention`` (split into partitions plus a merge when
    ``partition_size`` > 0).
 
-Host-to-device traffic of a step is the slot mapping, the copy pairs, the
-block tables and lengths, plus whatever the caller passes from host memory.
+Host-to-device traffic of a step is one small transfer: the slot mapping, the
+lengths, the table entries the reservation changed (at most one per row) and
+the copy pairs, plus whatever the caller passes from host memory.  The whole
+tables go over once, with ``upload_tables``.
 """
 
 import numpy as np
@@ -49,14 +51,41 @@ class PagedKVCache:
         self._h_slots = torch.empty(num_seqs, dtype=torch.int64).pin_memory()
         self._h_pairs = torch.empty((max(num_seqs, 1), 2), dtype=torch.int32).pin_memory()
         self.d_tables = torch.empty((num_seqs, self.max_blocks), dtype=torch.int32, device=self.device)
-        self.d_lens = torch.empty(num_seqs, dtype=torch.int32, device=self.device)
+        self._d_lens_full = torch.empty(num_seqs, dtype=torch.int32, device=self.device)
+        self.d_lens = self._d_lens_full     # after a decode_step: that step's lengths in its metadata slot
         self.d_slots = torch.empty(num_seqs, dtype=torch.int64, device=self.device)
         self.d_pairs = torch.empty((max(num_seqs, 1), 2), dtype=torch.int32, device=self.device)
         self._staged = None               # event: last copies out of the pinned staging buffers
+        # per-step metadata, double-buffered: [slots int64 S][lens int32 S][updates int32 S x 3][pairs int32 S x 2]
+        n = max(num_seqs, 1)
+        self._meta_bytes = 8 * n + 4 * n + 12 * n + 8 * n
+        self._meta_host = [torch.empty(self._meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self._meta_dev = [torch.empty(self._meta_bytes, dtype=torch.uint8, device=self.device) for _ in range(2)]
+        self._meta_done = [None, None]    # event: the H2D out of host slot b has finished
+        self._meta_views = [self._views(self._meta_host[b]) for b in range(2)]
+        self._meta_dviews = [self._views(self._meta_dev[b]) for b in range(2)]
+        self._step = 0
 
     @property
     def num_seqs(self):
         return self.lens.size
+
+    @property
+    def step_metadata_bytes(self):
+        """Bytes ``decode_step`` sends host -> device besides the caller's tensors."""
+        return self._meta_bytes
+
+    def _views(self, buf):
+        n = max(self.lens.size, 1)
+        o = 0
+        slots = buf[o:o + 8 * n].view(torch.int64)
+        o += 8 * n
+        lens = buf[o:o + 4 * n].view(torch.int32)
+        o += 4 * n
+        upd = buf[o:o + 12 * n].view(torch.int32).view(n, 3)
+        o += 12 * n
+        pairs = buf[o:o + 8 * n].view(torch.int32).view(n, 2)
+        return slots, lens, upd, pairs
 
     # ---------------------------------------------------------------- host side
 
@@ -82,14 +111,16 @@ class PagedKVCache:
         self.lens[row] = 0
 
     def reserve(self, rows=None):
-        """Reserve one slot in each of ``rows`` (a contiguous range ``slice`` or None = all)."""
+        """Reserve one slot in each of ``rows`` (a contiguous range ``slice`` or None = all).
+
+        Works in place on the host tables and lengths (a row range of a
+        C-contiguous array is itself contiguous).
+        """
         rows = slice(None) if rows is None else rows
-        tables = np.ascontiguousarray(self.tables[rows])
-        lens = np.ascontiguousarray(self.lens[rows])
-        slots, pairs = self.pool.pa_reserve_slots(tables, lens)
-        self.tables[rows] = tables
-        self.lens[rows] = lens
-        return slots, pairs
+        tables = self.tables[rows]
+        lens = self.lens[rows]
+        assert tables.flags.c_contiguous and lens.flags.c_contiguous
+        return self.pool.pa_reserve_slots(tables, lens)
 
     def _wait_staging(self):
         # the pinned buffers may still be read by an earlier asynchronous copy
@@ -106,6 +137,7 @@ class PagedKVCache:
         self._wait_staging()
         self._h_tables.numpy()[:] = self.tables
         self._h_lens.numpy()[:] = self.lens
+        self.d_lens = self._d_lens_full
         with torch.cuda.stream(stream):
             self.d_tables.copy_(self._h_tables, non_blocking=True)
             self.d_lens.copy_(self._h_lens, non_blocking=True)
@@ -129,25 +161,52 @@ class PagedKVCache:
         """One decode step for ``rows`` (default all): reserve, copy-on-write, append, attend.
 
         ``q``/``out`` cover the rows ([B, Hq, D]); ``k_new``/``v_new`` hold one
-        token per row ([B, Hkv, D]); all are CUDA tensors.  Returns the host
-        slot mapping and copy-on-write pairs of the step.
+        token per row ([B, Hkv, D]); all are CUDA tensors.  The host
+        reservation changes at most one table entry per row; those entries,
+        the slot mapping, the lengths and the copy pairs go to the device in
+        one small transfer, and ``pa_update_block_tables`` applies the entries
+        (the device tables must have been uploaded once with
+        ``upload_tables``).  Returns the host slot mapping and copy pairs.
         """
         stream = stream or torch.cuda.current_stream()
+        sel = slice(None) if rows is None else rows
+        r0 = sel.start or 0
+        lens_view = self.lens[sel]
+        tab_view = self.tables[sel]
+        n = lens_view.size
+        idx = np.arange(n)
+        cols = lens_view // self.block_size
+        old = tab_view[idx, np.minimum(cols, self.max_blocks - 1)].copy()
+        fresh = (lens_view % self.block_size) == 0
         slots, pairs = self.reserve(rows)
-        t = slots.size
-        self._wait_staging()
-        self._h_slots.numpy()[:t] = slots
+        new = tab_view[idx, cols]
+        changed = np.nonzero(fresh | (new != old))[0]
+        b = self._step & 1
+        self._step += 1
+        if self._meta_done[b] is not None:
+            self._meta_done[b].synchronize()          # the H2D out of this host slot has finished
+        h_slots, h_lens, h_upd, h_pairs = self._meta_views[b]
+        d_slots, d_lens, d_upd, d_pairs = self._meta_dviews[b]
+        h_slots.numpy()[:n] = slots
+        h_lens.numpy()[:self.lens.size] = self.lens
+        nu = changed.size
+        if nu:
+            u = h_upd.numpy()
+            u[:nu, 0] = changed + r0
+            u[:nu, 1] = cols[changed]
+            u[:nu, 2] = new[changed]
         npairs = pairs.shape[0]
         if npairs:
-            self._h_pairs.numpy()[:npairs] = pairs
+            h_pairs.numpy()[:npairs] = pairs
         with torch.cuda.stream(stream):
-            self.d_slots[:t].copy_(self._h_slots[:t], non_blocking=True)
-            if npairs:
-                self.d_pairs[:npairs].copy_(self._h_pairs[:npairs], non_blocking=True)
-        self.upload_tables(stream)
-        self.copy_blocks(self.d_pairs[:npairs], stream=stream)
-        self.append(k_new, v_new, self.d_slots[:t], stream=stream)
-        sel = slice(None) if rows is None else rows
-        self.attend(q, out, scale, partition_size, workspace, tables=self.d_tables[sel], lens=self.d_lens[sel],
+            self._meta_dev[b].copy_(self._meta_host[b], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            self._meta_done[b] = ev
+        self.d_lens = d_lens[:self.lens.size]          # the device lengths now live in this step's slot
+        pa.pa_update_block_tables(self.d_tables, d_upd[:nu], stream=stream)
+        self.copy_blocks(d_pairs[:npairs], stream=stream)
+        self.append(k_new, v_new, d_slots[:n], stream=stream)
+        self.attend(q, out, scale, partition_size, workspace, tables=self.d_tables[sel], lens=d_lens[sel],
                     stream=stream)
         return slots, pairs

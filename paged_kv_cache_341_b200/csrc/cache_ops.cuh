@@ -53,6 +53,23 @@ __global__ void __launch_bounds__(256) copy_kernel(uint4* k_cache, uint4* v_cach
   for (int i = begin + threadIdx.x; i < end; i += blockDim.x) d[i] = s[i];
 }
 
+// Block-table maintenance between steps: write the entries a host reservation
+// changed (a fresh block at a block boundary, or the copy of a shared block)
+// into the device tables, instead of re-sending whole tables.  updates[i] =
+// (row, column, block id); rows/columns outside the table are skipped and set
+// the device error word.
+__global__ void __launch_bounds__(256) table_update_kernel(int32_t* tables, int num_rows, int stride,
+                                                           const int32_t* __restrict__ updates, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int row = updates[3 * i], col = updates[3 * i + 1], val = updates[3 * i + 2];
+  if (row < 0 || row >= num_rows || col < 0 || col >= stride) {
+    set_device_error(DEVERR_BAD_SLOT);
+    return;
+  }
+  tables[static_cast<int64_t>(row) * stride + col] = val;
+}
+
 }  // namespace pa
 
 #endif

@@ -463,6 +463,20 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
   return pa::ok();
 }
 
+pa_status pa_update_block_tables(int32_t* block_tables, int32_t num_rows, int32_t table_stride,
+                                 const int32_t* updates, int32_t num_updates, void* stream) {
+  if (num_rows < 0 || table_stride <= 0 || num_updates < 0)
+    return pa::fail(PA_ERR_INVALID, "pa_update_block_tables: bad sizes");
+  if (num_updates == 0) return pa::ok();
+  if (!block_tables || !updates) return pa::fail(PA_ERR_INVALID, "pa_update_block_tables: null pointer");
+  const int threads = 256;
+  pa::table_update_kernel<<<(num_updates + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      block_tables, num_rows, table_stride, updates, num_updates);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "table_update_kernel launch");
+  return pa::ok();
+}
+
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
                                 int32_t block_size, int32_t partition_size) {
   if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||

@@ -46,6 +46,7 @@ SIGNATURES = {
     "pa_prefix_hash": (_i32, [_p32, _i32, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]),
     "pa_append_kv": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pa_update_block_tables": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp]),
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "pa_decode_attention": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
                                    _vp, _sz, _vp, _i32, _vp]),
@@ -246,6 +247,16 @@ def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
     _check(_lib.pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
                                _dev(pairs, "pairs", torch.int32), pairs.shape[0] if pairs.numel() else 0, nb, bs, hkv,
                                d, code, _stream(stream)))
+
+
+def pa_update_block_tables(block_tables, updates, stream=None):
+    """block_tables: int32 CUDA [rows, stride] (row-contiguous); updates: int32 CUDA [n, 3] (row, column, id)."""
+    if block_tables.dim() != 2 or block_tables.stride(1) != 1:
+        raise ValueError("block_tables must be a 2-D tensor with unit column stride")
+    n = updates.shape[0] if updates.numel() else 0
+    _check(_lib.pa_update_block_tables(ctypes.c_void_p(block_tables.data_ptr()), block_tables.shape[0],
+                                       block_tables.stride(0), _dev(updates, "updates", torch.int32) if n else None,
+                                       n, _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size):

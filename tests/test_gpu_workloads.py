@@ -84,6 +84,12 @@ def test_full_size_step(name):
     oracle_copy_blocks(sc.k_host, sc.v_host, opairs)
     oracle_append(sc.k_host, sc.v_host, k_new, v_new, oslots)
 
+    # the device tables followed the host reservation (entries applied incrementally)
+    for r in range(sc.rows.start, sc.rows.stop):
+        nblk = -(-olens[r] // w.block_size)
+        assert list(c.d_tables[r, :nblk].cpu().numpy()) == otables[r]
+    assert list(c.d_lens.cpu().numpy()) == olens
+
     # bit-exact: appended rows and copied blocks
     flat_k = c.k_cache.view(-1, w.num_kv_heads, w.head_dim)
     flat_v = c.v_cache.view(-1, w.num_kv_heads, w.head_dim)
