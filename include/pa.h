@@ -23,7 +23,9 @@
  * Conventions for every call:
  *   - Status codes only; nothing throws, aborts or traps.  On failure,
  *     pa_last_error() returns a message (per calling thread).
- *   - The library allocates NO device memory.  Caches, tables, workspace and
+ *   - Only pa_engine_create allocates (its own device staging, page-locked
+ *     host staging, streams and events, all freed by pa_engine_destroy); no
+ *     other call allocates device memory.  Caches, tables, workspace and
  *     outputs are device buffers owned by the caller (e.g. torch tensors'
  *     data_ptr()).  Host arrays are owned by the caller too.
  *   - Device calls are asynchronous on `stream` (a cudaStream_t; NULL is the
@@ -184,9 +186,13 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
  * boundary, or the private copy of a shared block), so sending the changes
  * instead of the tables keeps a step's host-to-device traffic small.
  * Out-of-range rows or columns are skipped and set the device error word (3).
- * Entries with the same (row, column) in one call must not repeat. */
+ * Entries with the same (row, column) in one call must not repeat.
+ * When context_lens (device int32 [num_rows]) is non-NULL, the same launch
+ * sets context_lens[i] = new_lens[i] for i < num_lens (device int32 array,
+ * num_lens <= num_rows); NULL context_lens skips the lengths. */
 pa_status pa_update_block_tables(int32_t* block_tables, int32_t num_rows, int32_t table_stride,
-                                 const int32_t* updates, int32_t num_updates, void* stream);
+                                 const int32_t* updates, int32_t num_updates, int32_t* context_lens,
+                                 const int32_t* new_lens, int32_t num_lens, void* stream);
 
 /* Bytes of device workspace pa_decode_attention takes for these sizes: 256
  * bytes for the work-unit counter, a planned work-unit list of 16 bytes per
@@ -312,6 +318,76 @@ pa_status pa_decode_attention_static(const void* q, const void* k_cache, const v
                                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                      int32_t head_dim, int32_t block_size, float scale,
                                      int32_t partition_size, void* out, pa_dtype dtype, void* stream);
+
+/* ---- Step executor ------------------------------------------------------
+ * One whole decode step of a batch, host buffers in and out, issued by one
+ * call: the slot reservation of pa_reserve_slots on the host, then on the
+ * GPU the table/length update (pa_update_block_tables), the copy-on-write
+ * copies (pa_copy_blocks), the append (pa_append_kv) and the attention
+ * (pa_decode_attention), with the host<->device copies around them
+ * (agentechip.com "Implementing a Simplified Paged KV Cache" and "Shared
+ * Prefix Caching"; krapton.com "How Paged Attention Works", steps 3-4).
+ *
+ * Copies run on two streams of the engine's own (upload, download) and the
+ * kernels on the caller's `stream`; the engine keeps two device slots for
+ * q, k_new, v_new, out and the step's metadata, so step i+1's upload and step
+ * i-1's download overlap step i's kernels.  Not thread-safe: one host thread
+ * drives an engine. */
+typedef struct pa_engine pa_engine;
+
+/* Create an engine for a batch of num_seqs sequences of one layer's cache.
+ * host_tables (int32 [num_seqs][max_blocks_per_seq]) and host_lens (int32
+ * [num_seqs]) are the caller's host block tables and lengths, and
+ * device_tables / device_lens the caller's device copies of them.  Each must
+ * already agree with the other before the first step (upload them once).
+ * k_cache / v_cache hold pool->num_blocks blocks of pool->block_size rows of
+ * [num_kv_heads][head_dim] elements of `dtype`.  All of them stay owned by
+ * the caller and must outlive the engine.  partition_size is passed to
+ * pa_decode_attention on every step (0 = single pass).  The engine allocates
+ * its staging (two slots of q, out, k_new, v_new and metadata, 32 bytes per
+ * sequence), the decode workspace, two streams and six events on the current
+ * device.  Errors: PA_ERR_INVALID for a bad argument (checked before anything
+ * is allocated), PA_ERR_CUDA when an allocation fails. */
+pa_status pa_engine_create(pa_pool* pool, int32_t* host_tables, int32_t* host_lens, int32_t num_seqs,
+                           int32_t max_blocks_per_seq, int32_t* device_tables, int32_t* device_lens,
+                           void* k_cache, void* v_cache, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, pa_dtype dtype, int32_t partition_size, void* stream,
+                           pa_engine** engine_out);
+
+/* Wait for everything the engine issued, then free what it allocated. */
+void pa_engine_destroy(pa_engine* engine);
+
+/* One decode step for rows [row0, row0 + num_rows) of the batch.
+ *   q      host [num_rows][num_q_heads][head_dim]   query of each row
+ *   k_new  host [num_rows][num_kv_heads][head_dim]  the new token's K
+ *   v_new  host [num_rows][num_kv_heads][head_dim]  the new token's V
+ *   out    host [num_rows][num_q_heads][head_dim]   attention output
+ * all of `dtype`, page-locked for the copies to overlap (pageable memory
+ * works, with copies that block the host).  The call reserves the slots
+ * (host tables and lengths change in place), enqueues the copies and kernels
+ * and returns without waiting for them.  The caller must leave q, k_new and
+ * v_new unchanged, and not read `out`, until the step is done: after the
+ * engine's next-but-one step returns, or after pa_engine_synchronize.  The
+ * new token attends to itself (it is appended before the attention).
+ * slots_out (host int64 [num_rows]) and pairs_out (host int32
+ * [num_rows][2]) receive the slot mapping and the copy-on-write pairs when
+ * non-NULL; num_pairs_out the number of pairs.  Errors: PA_ERR_INVALID for
+ * bad rows, buffers, scale or device; PA_ERR_EXHAUSTED when the pool runs
+ * dry (the pool, tables and lengths are then unchanged and nothing is
+ * enqueued); PA_ERR_CUDA when a copy or launch fails (the host reservation
+ * has then happened but the device state is undefined: destroy the engine
+ * and upload the tables again). */
+pa_status pa_engine_step(pa_engine* engine, int32_t row0, int32_t num_rows, const void* q,
+                         const void* k_new, const void* v_new, void* out, float scale,
+                         int64_t* slots_out, int32_t* pairs_out, int32_t* num_pairs_out);
+
+/* Make the caller's stream wait (on the device) for every copy the engine
+ * issued; the host does not block. */
+pa_status pa_engine_join(pa_engine* engine);
+
+/* Block the host until every step issued so far is done and its output is in
+ * host memory. */
+pa_status pa_engine_synchronize(pa_engine* engine);
 
 /* Read (and, if reset != 0, clear) the device error word of the current
  * device: 0 = none; 1 = block id outside the pool in a table; 2 =

@@ -23,7 +23,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v"]
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall"]
 SOURCES_CU = ["pa_device.cu"]
-SOURCES_CPP = ["pool.cpp", "prefix_cache.cpp", "common.cpp"]
+SOURCES_CPP = ["pool.cpp", "prefix_cache.cpp", "common.cpp", "engine.cpp"]
+CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 
 
 def nvcc():
@@ -64,7 +65,8 @@ def build(verbose=False):
         objs.append(obj)
     for src in SOURCES_CPP:
         obj = os.path.join(BUILD, src + ".o")
-        _run(["g++"] + CXX_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj], log)
+        _run(["g++"] + CXX_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-I", os.path.join(CUDA_HOME, "include"), "-c",
+                                   os.path.join(CSRC, src), "-o", obj], log)
         objs.append(obj)
     tmp = LIB + ".tmp"
     _run([nvcc()] + ARCH + ["-shared", "-o", tmp] + objs, log)

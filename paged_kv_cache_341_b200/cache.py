@@ -51,8 +51,7 @@ class PagedKVCache:
         self._h_slots = torch.empty(num_seqs, dtype=torch.int64).pin_memory()
         self._h_pairs = torch.empty((max(num_seqs, 1), 2), dtype=torch.int32).pin_memory()
         self.d_tables = torch.empty((num_seqs, self.max_blocks), dtype=torch.int32, device=self.device)
-        self._d_lens_full = torch.empty(num_seqs, dtype=torch.int32, device=self.device)
-        self.d_lens = self._d_lens_full     # after a decode_step: that step's lengths in its metadata slot
+        self.d_lens = torch.empty(num_seqs, dtype=torch.int32, device=self.device)
         self.d_slots = torch.empty(num_seqs, dtype=torch.int64, device=self.device)
         self.d_pairs = torch.empty((max(num_seqs, 1), 2), dtype=torch.int32, device=self.device)
         self._staged = None               # event: last copies out of the pinned staging buffers
@@ -137,7 +136,6 @@ class PagedKVCache:
         self._wait_staging()
         self._h_tables.numpy()[:] = self.tables
         self._h_lens.numpy()[:] = self.lens
-        self.d_lens = self._d_lens_full
         with torch.cuda.stream(stream):
             self.d_tables.copy_(self._h_tables, non_blocking=True)
             self.d_lens.copy_(self._h_lens, non_blocking=True)
@@ -203,10 +201,19 @@ class PagedKVCache:
             ev = torch.cuda.Event()
             ev.record(stream)
             self._meta_done[b] = ev
-        self.d_lens = d_lens[:self.lens.size]          # the device lengths now live in this step's slot
-        pa.pa_update_block_tables(self.d_tables, d_upd[:nu], stream=stream)
+        pa.pa_update_block_tables(self.d_tables, d_upd[:nu], self.d_lens, d_lens[:self.lens.size], stream=stream)
         self.copy_blocks(d_pairs[:npairs], stream=stream)
         self.append(k_new, v_new, d_slots[:n], stream=stream)
-        self.attend(q, out, scale, partition_size, workspace, tables=self.d_tables[sel], lens=d_lens[sel],
+        self.attend(q, out, scale, partition_size, workspace, tables=self.d_tables[sel], lens=self.d_lens[sel],
                     stream=stream)
         return slots, pairs
+
+    def engine(self, num_q_heads, partition_size=0, stream=None):
+        """A native step executor (``pa.Engine``) over this cache's pool, tables and lengths.
+
+        Uploads the tables and lengths first; afterwards steps go through the
+        engine (``pa_engine_step``, host buffers in and out).
+        """
+        self.upload_tables(stream)
+        return pa.Engine(self.pool, self.tables, self.lens, self.d_tables, self.d_lens, self.k_cache, self.v_cache,
+                         num_q_heads, partition_size, stream)

@@ -57,10 +57,14 @@ __global__ void __launch_bounds__(256) copy_kernel(uint4* k_cache, uint4* v_cach
 // changed (a fresh block at a block boundary, or the copy of a shared block)
 // into the device tables, instead of re-sending whole tables.  updates[i] =
 // (row, column, block id); rows/columns outside the table are skipped and set
-// the device error word.
+// the device error word.  The same launch copies the step's lengths into the
+// device lengths (lens[i] = new_lens[i], i < num_lens) when lens is non-null.
 __global__ void __launch_bounds__(256) table_update_kernel(int32_t* tables, int num_rows, int stride,
-                                                           const int32_t* __restrict__ updates, int n) {
+                                                           const int32_t* __restrict__ updates, int n,
+                                                           int32_t* lens, const int32_t* __restrict__ new_lens,
+                                                           int num_lens) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (lens != nullptr && i < num_lens) lens[i] = new_lens[i];
   if (i >= n) return;
   const int row = updates[3 * i], col = updates[3 * i + 1], val = updates[3 * i + 2];
   if (row < 0 || row >= num_rows || col < 0 || col >= stride) {

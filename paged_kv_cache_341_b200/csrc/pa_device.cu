@@ -464,14 +464,19 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
 }
 
 pa_status pa_update_block_tables(int32_t* block_tables, int32_t num_rows, int32_t table_stride,
-                                 const int32_t* updates, int32_t num_updates, void* stream) {
-  if (num_rows < 0 || table_stride <= 0 || num_updates < 0)
+                                 const int32_t* updates, int32_t num_updates, int32_t* context_lens,
+                                 const int32_t* new_lens, int32_t num_lens, void* stream) {
+  if (num_rows < 0 || table_stride <= 0 || num_updates < 0 || num_lens < 0 || num_lens > num_rows)
     return pa::fail(PA_ERR_INVALID, "pa_update_block_tables: bad sizes");
-  if (num_updates == 0) return pa::ok();
-  if (!block_tables || !updates) return pa::fail(PA_ERR_INVALID, "pa_update_block_tables: null pointer");
+  if (!context_lens) num_lens = 0;
+  const int n = num_updates > num_lens ? num_updates : num_lens;
+  if (n == 0) return pa::ok();
+  if ((num_updates > 0 && (!block_tables || !updates)) || (num_lens > 0 && !new_lens))
+    return pa::fail(PA_ERR_INVALID, "pa_update_block_tables: null pointer");
   const int threads = 256;
-  pa::table_update_kernel<<<(num_updates + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      block_tables, num_rows, table_stride, updates, num_updates);
+  pa::table_update_kernel<<<(n + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      block_tables, num_rows, table_stride, updates, num_updates, num_lens ? context_lens : nullptr, new_lens,
+      num_lens);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "table_update_kernel launch");
   return pa::ok();

@@ -46,7 +46,13 @@ SIGNATURES = {
     "pa_prefix_hash": (_i32, [_p32, _i32, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]),
     "pa_append_kv": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
-    "pa_update_block_tables": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp]),
+    "pa_update_block_tables": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
+    "pa_engine_create": (_i32, [_vp, _p32, _p32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                                ctypes.POINTER(_vp)]),
+    "pa_engine_destroy": (None, [_vp]),
+    "pa_engine_step": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp, _f32, _p64, _p32, _p32]),
+    "pa_engine_join": (_i32, [_vp]),
+    "pa_engine_synchronize": (_i32, [_vp]),
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "pa_decode_attention": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
                                    _vp, _sz, _vp, _i32, _vp]),
@@ -249,14 +255,20 @@ def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
                                d, code, _stream(stream)))
 
 
-def pa_update_block_tables(block_tables, updates, stream=None):
-    """block_tables: int32 CUDA [rows, stride] (row-contiguous); updates: int32 CUDA [n, 3] (row, column, id)."""
+def pa_update_block_tables(block_tables, updates, context_lens=None, new_lens=None, stream=None):
+    """block_tables: int32 CUDA [rows, stride] (row-contiguous); updates: int32 CUDA [n, 3] (row, column, id).
+
+    With ``context_lens`` (int32 CUDA [rows]) the same launch also sets
+    ``context_lens[:len(new_lens)] = new_lens``.
+    """
     if block_tables.dim() != 2 or block_tables.stride(1) != 1:
         raise ValueError("block_tables must be a 2-D tensor with unit column stride")
     n = updates.shape[0] if updates.numel() else 0
+    nl = 0 if context_lens is None else new_lens.numel()
     _check(_lib.pa_update_block_tables(ctypes.c_void_p(block_tables.data_ptr()), block_tables.shape[0],
                                        block_tables.stride(0), _dev(updates, "updates", torch.int32) if n else None,
-                                       n, _stream(stream)))
+                                       n, _dev(context_lens, "context_lens", torch.int32) if nl else None,
+                                       _dev(new_lens, "new_lens", torch.int32) if nl else None, nl, _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size):
@@ -358,3 +370,81 @@ def pa_device_error(reset=True):
     code = ctypes.c_int32()
     _check(_lib.pa_device_error(ctypes.byref(code), 1 if reset else 0))
     return code.value
+
+
+# --------------------------------------------------------------------------
+# Step executor
+# --------------------------------------------------------------------------
+
+def _host(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError("%s must be a host (CPU) tensor" % name)
+    if not t.is_contiguous() or t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must be a contiguous %s tensor of shape %s" % (name, dtype, tuple(shape)))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Engine:
+    """pa_engine_*: one decode step of a batch per call, host buffers in and out.
+
+    ``host_tables`` / ``host_lens`` are the caller's numpy int32 arrays
+    ([S, max_blocks], [S]), changed in place by every step; ``device_tables``
+    / ``device_lens`` their CUDA copies (already uploaded).  The engine keeps
+    references to all of them so they outlive it.
+    """
+
+    def __init__(self, pool, host_tables, host_lens, device_tables, device_lens, k_cache, v_cache, num_q_heads,
+                 partition_size=0, stream=None):
+        if host_tables.dtype != np.int32 or not host_tables.flags.c_contiguous or host_tables.ndim != 2:
+            raise TypeError("host_tables must be a C-contiguous int32 [S, max_blocks] array")
+        if host_lens.dtype != np.int32 or not host_lens.flags.c_contiguous or host_lens.size != host_tables.shape[0]:
+            raise TypeError("host_lens must be a contiguous int32 [S] array")
+        nb, bs, hkv, d = k_cache.shape
+        s, mb = host_tables.shape
+        if tuple(device_tables.shape) != (s, mb) or device_lens.numel() != s:
+            raise ValueError("device tables/lengths must match the host ones")
+        self._keep = (pool, host_tables, host_lens, device_tables, device_lens, k_cache, v_cache)
+        self._stream = stream if stream is not None else torch.cuda.current_stream()
+        self.dtype = k_cache.dtype
+        self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, hkv, d
+        handle = ctypes.c_void_p()
+        _check(_lib.pa_engine_create(pool._h, host_tables.ctypes.data_as(_p32), host_lens.ctypes.data_as(_p32), s,
+                                     mb, _dev(device_tables, "device_tables", torch.int32),
+                                     _dev(device_lens, "device_lens", torch.int32), _dev(k_cache, "k_cache"),
+                                     _dev(v_cache, "v_cache", k_cache.dtype), num_q_heads, hkv, d,
+                                     DTYPE_CODE[k_cache.dtype], partition_size, _stream(self._stream),
+                                     ctypes.byref(handle)))
+        self._h = handle
+        self._slots = np.empty(s, np.int64)
+        self._pairs = np.empty((s, 2), np.int32)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.pa_engine_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def pa_engine_step(self, row0, num_rows, q, k_new, v_new, out, scale, want_slots=False):
+        """Enqueue one step; returns (slots, pairs) copies when ``want_slots`` else the pair count."""
+        hq, hkv, d = self.num_q_heads, self.num_kv_heads, self.head_dim
+        npairs = ctypes.c_int32()
+        _check(_lib.pa_engine_step(self._h, row0, num_rows, _host(q, "q", self.dtype, (num_rows, hq, d)),
+                                   _host(k_new, "k_new", self.dtype, (num_rows, hkv, d)),
+                                   _host(v_new, "v_new", self.dtype, (num_rows, hkv, d)),
+                                   _host(out, "out", self.dtype, (num_rows, hq, d)), scale,
+                                   self._slots.ctypes.data_as(_p64) if want_slots else None,
+                                   self._pairs.ctypes.data_as(_p32) if want_slots else None, ctypes.byref(npairs)))
+        if want_slots:
+            return self._slots[:num_rows].copy(), self._pairs[:npairs.value].copy()
+        return npairs.value
+
+    def pa_engine_join(self):
+        _check(_lib.pa_engine_join(self._h))
+
+    def pa_engine_synchronize(self):
+        _check(_lib.pa_engine_synchronize(self._h))

@@ -93,3 +93,46 @@ def test_binding_refuses_cpu_tensors(built_library):
         pa.pa_decode_attention(x, torch.zeros(16, 16, 2, 64), torch.zeros(16, 16, 2, 64),
                                torch.zeros(4, 4, dtype=torch.int32), torch.zeros(4, dtype=torch.int32), 0.125,
                                torch.zeros(4, 2, 64))
+
+
+def test_table_update_and_engine_reject_bad_arguments_on_host(built_library):
+    import numpy as np
+    from paged_kv_cache_341_b200 import pa
+    lib = pa._lib
+    fake = ctypes.c_void_p(1 << 20)
+    # nothing to do -> OK without touching the device; bad sizes -> INVALID
+    assert lib.pa_update_block_tables(fake, 4, 8, fake, 0, None, None, 0, None) == pa.PA_OK
+    assert lib.pa_update_block_tables(fake, 4, 0, fake, 1, None, None, 0, None) == pa.PA_ERR_INVALID
+    assert lib.pa_update_block_tables(fake, 4, 8, fake, 1, fake, fake, 5, None) == pa.PA_ERR_INVALID
+    assert lib.pa_update_block_tables(None, 4, 8, None, 2, None, None, 0, None) == pa.PA_ERR_INVALID
+
+    pool = pa.Pool(16, 16)
+    tables = np.zeros((2, 4), np.int32)
+    lens = np.zeros(2, np.int32)
+    t32 = tables.ctypes.data_as(pa._p32)
+    l32 = lens.ctypes.data_as(pa._p32)
+    out = ctypes.c_void_p(123)
+
+    def create(**kw):
+        a = dict(pool=pool._h, tables=t32, lens=l32, s=2, mb=4, dt=fake, dl=fake, k=fake, v=fake, hq=4, hkv=2,
+                 d=64, dtype=pa.PA_BF16, part=0)
+        a.update(kw)
+        return lib.pa_engine_create(a["pool"], a["tables"], a["lens"], a["s"], a["mb"], a["dt"], a["dl"], a["k"],
+                                    a["v"], a["hq"], a["hkv"], a["d"], a["dtype"], a["part"], None,
+                                    ctypes.byref(out))
+
+    # every argument check runs before anything is allocated on the device
+    assert create(pool=None) == pa.PA_ERR_INVALID and out.value is None
+    assert create(s=0) == pa.PA_ERR_INVALID
+    assert create(hq=3) == pa.PA_ERR_INVALID
+    assert create(dtype=7) == pa.PA_ERR_INVALID
+    assert create(k=ctypes.c_void_p((1 << 20) + 8)) == pa.PA_ERR_INVALID
+    assert create(part=24) == pa.PA_ERR_INVALID
+    assert create(part=-16) == pa.PA_ERR_INVALID
+    assert lib.pa_engine_create(pool._h, t32, l32, 2, 4, fake, fake, fake, fake, 4, 2, 64, pa.PA_BF16, 0, None,
+                                None) == pa.PA_ERR_INVALID
+    assert lib.pa_engine_step(None, 0, 1, fake, fake, fake, fake, 1.0, None, None, None) == pa.PA_ERR_INVALID
+    assert lib.pa_engine_join(None) == pa.PA_ERR_INVALID
+    assert lib.pa_engine_synchronize(None) == pa.PA_ERR_INVALID
+    lib.pa_engine_destroy(None)
+    assert "pa_engine" in pa.pa_last_error()
