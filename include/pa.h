@@ -319,6 +319,14 @@ pa_status pa_decode_attention_static(const void* q, const void* k_cache, const v
                                      int32_t head_dim, int32_t block_size, float scale,
                                      int32_t partition_size, void* out, pa_dtype dtype, void* stream);
 
+/* Practical read-bandwidth ceiling (a measurement aid, not a step of the
+ * path): read every byte of `buf` (device, 16-byte aligned, `bytes` a
+ * multiple of 16) once with streaming 16-byte loads on a grid of 4 CTAs of
+ * 512 threads per SM, and XOR-fold what was read into *sink (device uint32).
+ * Timing it on a buffer larger than L2 gives the bandwidth a read-only
+ * stream such as decode attention can reach on this GPU. */
+pa_status pa_read_stream(const void* buf, size_t bytes, uint32_t* sink, void* stream);
+
 /* ---- Step executor ------------------------------------------------------
  * One whole decode step of a batch, host buffers in and out, issued by one
  * call: the slot reservation of pa_reserve_slots on the host, then on the

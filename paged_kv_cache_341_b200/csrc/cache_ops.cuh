@@ -74,6 +74,28 @@ __global__ void __launch_bounds__(256) table_update_kernel(int32_t* tables, int 
   tables[static_cast<int64_t>(row) * stride + col] = val;
 }
 
+// Read-bandwidth ceiling: every byte of a buffer read once with streaming
+// (evict-first) 16-byte loads, four in flight per thread, XOR-folded so the
+// loads cannot be dropped.  No writes apart from one word per warp.  The
+// decode kernel's achieved bandwidth is compared against this as the
+// practical ceiling of a read-only stream on the GPU at hand.
+__global__ void __launch_bounds__(512, 4) read_stream_kernel(const uint4* __restrict__ p, int64_t n, uint32_t* sink) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t acc = 0;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    const uint4 a = __ldcs(p + i), b = __ldcs(p + i + stride), c = __ldcs(p + i + 2 * stride),
+                d = __ldcs(p + i + 3 * stride);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w ^ c.x ^ c.y ^ c.z ^ c.w ^ d.x ^ d.y ^ d.z ^ d.w;
+  }
+  for (; i < n; i += stride) {
+    const uint4 a = __ldcs(p + i);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  }
+  for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) atomicXor(sink, acc);
+}
+
 }  // namespace pa
 
 #endif

@@ -482,6 +482,20 @@ pa_status pa_update_block_tables(int32_t* block_tables, int32_t num_rows, int32_
   return pa::ok();
 }
 
+pa_status pa_read_stream(const void* buf, size_t bytes, uint32_t* sink, void* stream) {
+  if (bytes % 16 != 0) return pa::fail(PA_ERR_INVALID, "pa_read_stream: bytes must be a multiple of 16");
+  if (bytes == 0) return pa::ok();
+  if (!buf || !sink || !aligned16(buf)) return pa::fail(PA_ERR_INVALID, "pa_read_stream: null or misaligned buffer");
+  DeviceInfo di;
+  pa_status st = device_info(&di);
+  if (st != PA_OK) return st;
+  pa::read_stream_kernel<<<di.sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(buf), static_cast<int64_t>(bytes / 16), sink);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "read_stream_kernel launch");
+  return pa::ok();
+}
+
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
                                 int32_t block_size, int32_t partition_size) {
   if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||

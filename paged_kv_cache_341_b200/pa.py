@@ -47,6 +47,7 @@ SIGNATURES = {
     "pa_append_kv": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_update_block_tables": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
+    "pa_read_stream": (_i32, [_vp, _sz, _vp, _vp]),
     "pa_engine_create": (_i32, [_vp, _p32, _p32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
                                 ctypes.POINTER(_vp)]),
     "pa_engine_destroy": (None, [_vp]),
@@ -269,6 +270,12 @@ def pa_update_block_tables(block_tables, updates, context_lens=None, new_lens=No
                                        block_tables.stride(0), _dev(updates, "updates", torch.int32) if n else None,
                                        n, _dev(context_lens, "context_lens", torch.int32) if nl else None,
                                        _dev(new_lens, "new_lens", torch.int32) if nl else None, nl, _stream(stream)))
+
+
+def pa_read_stream(buf, sink, stream=None):
+    """Read all of ``buf`` (CUDA tensor, contiguous) once; XOR of what was read lands in ``sink`` (int32 CUDA [1])."""
+    _check(_lib.pa_read_stream(_dev(buf, "buf"), buf.numel() * buf.element_size(), _dev(sink, "sink", torch.int32),
+                               _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_size):
