@@ -13,6 +13,7 @@
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "prefix.cuh"
+#include "prefix_tc.cuh"
 #include "pa.h"
 #include "pa_common.h"
 
@@ -344,11 +345,65 @@ struct PrefixArgs {
   int prefix_len;
 };
 
+// Prefix kernel: tcgen05 (tensor memory) by default; PA_PREFIX_PATH=mma picks
+// the mma.sync kernel (same results within rounding, kept for comparison).
+bool prefix_uses_umma() {
+  const char* v = std::getenv("PA_PREFIX_PATH");
+  return !(v && std::string(v) == "mma");
+}
+
+template <typename T, int D, int G>
+pa_status launch_prefix_umma(const DecodeArgs& a, const PrefixArgs& pf, const DeviceInfo& dev) {
+  int stages = 4;
+  const int forced_st = env_int("PA_PREFIX_STAGES");
+  if (forced_st >= 2 && forced_st <= 6) stages = forced_st;
+  while (stages >= 2 && pa::prefix_umma_smem_bytes<D>(stages) > static_cast<size_t>(dev.smem_optin)) --stages;
+  if (stages < 2) return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: stage does not fit in shared memory");
+  const size_t smem = pa::prefix_umma_smem_bytes<D>(stages);
+  auto kern = pa::prefix_umma_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix umma)");
+  CUtensorMap tm_k, tm_v;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
+  const int box_rows = a.BS < pa::kChunkTokens ? a.BS : pa::kChunkTokens;
+  pa_status st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  const int np = a.total_parts;
+  const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
+  char* ws = static_cast<char*>(a.workspace);
+  const size_t list_bytes = units_bytes(a.S, a.Hq, max_parts(a.max_blocks, a.BS, a.P));
+  pa::PrefixParams prm;
+  prm.q = a.q;
+  prm.prefix_blocks = pf.prefix_blocks;
+  prm.part_acc = reinterpret_cast<float*>(ws + kSchedBytes + list_bytes);
+  prm.part_ml = reinterpret_cast<float2*>(prm.part_acc + acc_elems);
+  prm.num_seqs = a.S;
+  prm.num_q_heads = a.Hq;
+  prm.num_kv_heads = a.Hkv;
+  prm.block_size = a.BS;
+  prm.num_blocks = a.num_blocks;
+  prm.prefix_len = pf.prefix_len;
+  prm.split_tokens = kPrefixSplitTokens;
+  prm.max_parts = np;
+  prm.stages = stages;
+  prm.stage_bytes = static_cast<uint32_t>(pa::kUmmaTile * D * sizeof(T));
+  prm.qk_scale = a.scale * 1.4426950408889634f;
+  constexpr int kCtaRows = pa::kUmmaTiles * pa::kUmmaRows;
+  const dim3 grid((a.S * G + kCtaRows - 1) / kCtaRows, a.Hkv, prefix_splits(pf.prefix_len));
+  kern<<<grid, pa::kUmmaThreads, smem, a.stream>>>(tm_k, tm_v, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefix_umma_kernel launch");
+  return PA_OK;
+}
+
 template <typename T, int D, int G>
 pa_status launch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   DeviceInfo dev;
   pa_status st = device_info(&dev);
   if (st != PA_OK) return st;
+  if (prefix_uses_umma()) return launch_prefix_umma<T, D, G>(a, pf, dev);
   const size_t stage_bytes = static_cast<size_t>(pa::kPrefixTile) * D * sizeof(T);
   int stages = 3;
   const int forced_st = env_int("PA_PREFIX_STAGES");

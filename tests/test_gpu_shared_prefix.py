@@ -26,7 +26,14 @@ def pa():
     return mod
 
 
-def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed):
+@pytest.fixture(params=["umma", "mma"])
+def prefix_path(request, monkeypatch):
+    """Run a test once on the tcgen05 (tensor-memory) prefix kernel and once on the mma.sync one."""
+    monkeypatch.setenv("PA_PREFIX_PATH", request.param)
+    return request.param
+
+
+def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed, q_scale=1.0):
     from paged_kv_cache_341_b200.cache import PagedKVCache
     rng = np.random.default_rng(seed)
     s = len(suffixes)
@@ -48,6 +55,8 @@ def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed
     cache.v_cache.copy_(v_host)
     cache.upload_tables()
     q_host = workloads.randn((s, hq, d), dtype, seed + 2)
+    if q_scale != 1.0:
+        q_host = (q_host.float() * q_scale).to(TORCH[dtype])
     q = q_host.cuda()
     scale = 1.0 / math.sqrt(d)
     out = torch.full((s, hq, d), float("nan"), dtype=TORCH[dtype], device="cuda")
@@ -74,21 +83,33 @@ SUFFIXES = [0, 1, 15, 16, 17, 100, 33]
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (16, 4), (16, 2)])
 @pytest.mark.parametrize("bs", [8, 16, 32])
-@pytest.mark.parametrize("prefix_len", [32, 1088])
+@pytest.mark.parametrize("prefix_len", [32, 1056, 1088])
 @pytest.mark.parametrize("partition", [0, 64])
-def test_shared_prefix_matches_oracle(pa, dtype, d, hq, hkv, bs, prefix_len, partition):
+def test_shared_prefix_matches_oracle(pa, prefix_path, dtype, d, hq, hkv, bs, prefix_len, partition):
+    # 1056 = 1024 + 32: the second slice ends in a 32-token tile; 1088 ends on a full one
     gpu, ref, plain = run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, SUFFIXES, partition,
                                   seed=prefix_len + bs + hq + d + partition)
-    tag = "dtype=%s d=%d hq=%d hkv=%d bs=%d prefix=%d p=%d" % (dtype, d, hq, hkv, bs, prefix_len, partition)
+    tag = "%s dtype=%s d=%d hq=%d hkv=%d bs=%d prefix=%d p=%d" % (prefix_path, dtype, d, hq, hkv, bs, prefix_len,
+                                                                  partition)
     assert_close(gpu, ref, dtype, tag)
     assert_close(gpu, plain.astype(np.float64), dtype, tag + " vs plain call")
 
 
-def test_many_sequences_and_row_tiles(pa):
+@pytest.mark.parametrize("nseq", [70, 50, 64])
+def test_many_sequences_and_row_tiles(pa, prefix_path, nseq):
+    # x 4 query rows per KV head: 280 = tiles of 128, 128 and 24; 200 = 128 and
+    # 72 (a partly filled second tile of a CTA); 256 = exactly two full tiles
     rng = np.random.default_rng(5)
-    suffixes = [int(x) for x in rng.integers(0, 600, size=70)]
-    gpu, ref, _ = run_cascade(pa, "bf16", 32, 8, 128, 16, 2048 + 64, suffixes, 512, seed=6)
-    assert_close(gpu, ref, "bf16", "70 sequences")
+    suffixes = [int(x) for x in rng.integers(0, 600, size=nseq)]
+    gpu, ref, _ = run_cascade(pa, "bf16", 32, 8, 128, 16, 2048 + 64, suffixes, 512, seed=6 + nseq)
+    assert_close(gpu, ref, "bf16", "%d sequences" % nseq)
+
+
+def test_large_scores_rescale_in_tensor_memory(pa, prefix_path):
+    # queries scaled up so the running maximum moves by more than 2^8 between
+    # tiles: the tcgen05 kernel rescales O inside tensor memory
+    gpu, ref, _ = run_cascade(pa, "bf16", 16, 4, 128, 16, 1024 + 512, [3, 0, 40], 0, seed=8, q_scale=12.0)
+    assert_close(gpu, ref, "bf16", "large scores")
 
 
 def test_zero_prefix_is_the_plain_call(pa):
