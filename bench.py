@@ -379,22 +379,22 @@ def run_ours(args):
     ms, att_ms = max_over_ranks([ms, att_ms], device="cuda")
     assert pa.pa_device_error() == 0
 
-    # ---- practical read ceiling: the K and V pools (each larger than L2) read
-    # once each with streaming loads, same GPU, right after the timed region
+    # ---- practical read ceiling: a dedicated 2 GiB buffer (16x L2) read once
+    # per pass with streaming loads, same GPU, right after the timed region
+    read_buf = torch.ones(1 << 29, dtype=torch.int32, device="cuda")
     sink = torch.zeros(1, dtype=torch.int32, device="cuda")
     for _ in range(3):
-        pa.pa_read_stream(c.k_cache, sink)
-        pa.pa_read_stream(c.v_cache, sink)
+        pa.pa_read_stream(read_buf, sink)
     r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_read = 20
     r0.record(stream)
     for _ in range(n_read):
-        pa.pa_read_stream(c.k_cache, sink)
-        pa.pa_read_stream(c.v_cache, sink)
+        pa.pa_read_stream(read_buf, sink)
     r1.record(stream)
     torch.cuda.synchronize()
-    read_bytes = 2 * c.k_cache.numel() * c.k_cache.element_size()
+    read_bytes = read_buf.numel() * read_buf.element_size()
     read_gbs = read_bytes * n_read / (r0.elapsed_time(r1) / 1e3) / 1e9
+    del read_buf
 
     # ---- end to end through the public API from pinned host memory: one
     # pa_engine_step call per step does the host slot reservation, the H2D of
@@ -476,9 +476,8 @@ def run_ours(args):
                                        n_att, peak_kind),
                          "algorithmic_bytes_per_launch": kv_bytes,
                          "read_ceiling": {"value": round(read_gbs, 2), "unit": "GB/s",
-                                          "kernel": "read_stream_kernel (pa_read_stream): K and V pools, %.2f GB, "
-                                                    "read once per pass, mean of %d passes" % (read_bytes / 1e9,
-                                                                                             n_read)},
+                                          "kernel": "read_stream_kernel (pa_read_stream): %.2f GB buffer read once "
+                                                    "per pass, mean of %d passes" % (read_bytes / 1e9, n_read)},
                          "frac_of_read_ceiling": round(achieved / read_gbs, 4)},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,

@@ -83,7 +83,7 @@ def build(verbose=False):
 def kernel_digest():
     """Digest of the decode kernel's sources and launch code (ties ncu counters to the code they were taken on)."""
     h = hashlib.sha256()
-    for name in ("decode.cuh", "ptx.cuh", "dtype.cuh", "pa_device.cu"):
+    for name in ("decode.cuh", "ptx.cuh", "dtype.cuh", "launch_decode.cuh"):
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
