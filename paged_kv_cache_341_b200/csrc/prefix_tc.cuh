@@ -46,6 +46,17 @@
 
 namespace pa {
 
+// d += a on a pair of float32 lanes (one instruction on sm_100a).
+__device__ __forceinline__ void fadd2(float2& d, const float2 a) {
+  asm("{\n\t.reg .b64 rd, ra;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(a.x), "f"(a.y));
+}
+
 constexpr int kUmmaRows = 128;        // query rows per tile (MMA M)
 constexpr int kUmmaTiles = 2;         // query tiles per CTA
 constexpr int kUmmaTile = 64;         // prefix tokens per stage (MMA N of S, K of O)
@@ -237,10 +248,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_f16<kBf16>(kUmmaRows, kUmmaTile, false, false);
       constexpr uint32_t idesc_o = tc::idesc_f16<kBf16>(kUmmaRows, D, false, true);
-      const uint32_t q_addr = smem_addr(s_q);
-      const uint32_t p_addr = smem_addr(s_p);
-      const uint32_t k_addr = smem_addr(s_k);
-      const uint32_t v_addr = smem_addr(s_v);
+      // descriptors of the operand bases; an operand at byte offset x from a
+      // base is the base descriptor plus x >> 4 (start-address field, no carry
+      // below 256 KB of shared memory)
+      const uint64_t q_desc = tc::smem_desc_sw128(smem_addr(s_q), 16, 1024);
+      const uint64_t p_desc = tc::smem_desc_sw128(smem_addr(s_p), 16, 1024);
+      const uint64_t k_desc = tc::smem_desc_sw128(smem_addr(s_k), 16, 1024);
+      const uint64_t v_desc = tc::smem_desc_sw128(smem_addr(s_v), kPanel, 1024);
       int kst = 0, vst = 0;
       uint32_t kph = 0, vph = 0;
       bool ok = true;
@@ -248,17 +262,15 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       tc::fence_after_sync();
       auto pv = [&](int j) -> bool {
         if (!mbar_wait(&v_full[vst], vph, abort_flag)) return false;
-        const uint32_t vb = v_addr + vst * kTileBytes;
+        const uint64_t vb = v_desc + ((vst * kTileBytes) >> 4);
         for (int g = 0; g < ngroups; ++g) {
           if (!mbar_wait(p_full(g, j & 1), (j >> 1) & 1, abort_flag)) return false;
           tc::fence_after_sync();
-          const uint32_t pb = p_addr + (2 * g + (j & 1)) * kPBytes;
+          const uint64_t pb = p_desc + (((2 * g + (j & 1)) * kPBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kUmmaTile / 16; ++kk) {
-            const uint64_t a = tc::smem_desc_sw128(pb + kk * 32, 16, 1024);
-            const uint64_t b = tc::smem_desc_sw128(vb + kk * 16 * 128, kPanel, 1024);
-            tc::mma_f16_ss(tmem + g * 256 + 128, a, b, idesc_o, j > 0 || kk > 0);
-          }
+          for (int kk = 0; kk < kUmmaTile / 16; ++kk)
+            tc::mma_f16_ss(tmem + g * 256 + 128, pb + ((kk * 32) >> 4), vb + ((kk * 16 * 128) >> 4), idesc_o,
+                           j > 0 || kk > 0);
           tc::commit(pv_done(g, j & 1));
         }
         tc::commit(&v_empty[vst]);
@@ -274,20 +286,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t kb = k_addr + kst * kTileBytes;
+        const uint64_t kb = k_desc + ((kst * kTileBytes) >> 4);
         for (int g = 0; g < ngroups && ok; ++g) {
           if (t >= 2 && !mbar_wait(s_free(g, sb), ((t - 2) >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
+          const uint64_t qb = q_desc + ((g * kQBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a =
-                tc::smem_desc_sw128(q_addr + g * kQBytes + (kk >> 2) * kQPanel + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = tc::smem_desc_sw128(kb + (kk >> 2) * kPanel + (kk & 3) * 32, 16, 1024);
-            tc::mma_f16_ss(tmem + g * 256 + sb * kUmmaTile, a, b, idesc_s, kk > 0);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc::mma_f16_ss(tmem + g * 256 + sb * kUmmaTile, qb + (((kk >> 2) * kQPanel + (kk & 3) * 32) >> 4),
+                           kb + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
           tc::commit(s_full(g, sb));
         }
         if (!ok) break;
@@ -345,34 +355,59 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free(g, sb));
-      float x[kUmmaTile];
+      // raw scores; the scaled maximum is max(s) * qk for qk >= 0 and
+      // min(s) * qk otherwise (rounding is monotonic, so this equals the
+      // maximum of the rounded products); columns past a short last tile
+      // never win and get weight 0
+      const float qk = prm.qk_scale;
+      const bool full = ntok == kUmmaTile;
+      float sv[kUmmaTile];
 #pragma unroll
-      for (int j = 0; j < kUmmaTile; ++j)
-        x[j] = j < ntok ? __uint_as_float(sr[j >> 5][j & 31]) * prm.qk_scale : -INFINITY;
-      // row maximum as a tree (8 independent chains)
+      for (int j = 0; j < kUmmaTile; ++j) sv[j] = __uint_as_float(sr[j >> 5][j & 31]);
+      const float pad = qk >= 0.f ? -INFINITY : INFINITY;
+      if (!full) {
+#pragma unroll
+        for (int j = 0; j < kUmmaTile; ++j) sv[j] = j < ntok ? sv[j] : pad;
+      }
       float cm[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cm[i] = x[i];
+      for (int i = 0; i < 8; ++i) cm[i] = sv[i];
+      if (qk >= 0.f) {
 #pragma unroll
-      for (int j = 8; j < kUmmaTile; ++j) cm[j & 7] = fmaxf(cm[j & 7], x[j]);
-      const float c = fmaxf(fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])),
-                            fmaxf(fmaxf(cm[4], cm[5]), fmaxf(cm[6], cm[7])));
-      const float mn = c > m + kTau ? c : m;
-      // P row: 64 weights relative to the new reference, rounded to T; the
-      // row sum of the rounded weights in 8 independent chains
-      uint32_t w[kUmmaTile / 2];
-      float ls[8];
+        for (int j = 8; j < kUmmaTile; ++j) cm[j & 7] = fmaxf(cm[j & 7], sv[j]);
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        ls[ch] = 0.f;
+        for (int i = 0; i < 4; ++i) cm[i] = fmaxf(cm[i], cm[i + 4]);
+        cm[0] = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+      } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int j = ch * 8 + 2 * k;
-          w[ch * 4 + k] = M::pack(exp2_approx(x[j] - mn), exp2_approx(x[j + 1] - mn));
-          const float2 u = M::unpack(w[ch * 4 + k]);
-          ls[ch] += u.x + u.y;
-        }
+        for (int j = 8; j < kUmmaTile; ++j) cm[j & 7] = fminf(cm[j & 7], sv[j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cm[i] = fminf(cm[i], cm[i + 4]);
+        cm[0] = fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
       }
+      const float c = cm[0] * qk;
+      const float mn = c > m + kTau ? c : m;
+      // P row: 2^(s*qk - m) with one packed FMA per pair, rounded to T; the
+      // row sum of the rounded weights with packed adds in 4 chains
+      uint32_t w[kUmmaTile / 2];
+      float2 ls[4];
+      const float2 qk2 = make_float2(qk, qk);
+      const float2 nm2 = make_float2(-mn, -mn);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ls[k] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < kUmmaTile / 2; ++i) {
+        float2 e = nm2;
+        ffma2(e, make_float2(sv[2 * i], sv[2 * i + 1]), qk2);
+        float p0 = exp2_approx(e.x), p1 = exp2_approx(e.y);
+        if (!full) {
+          p0 = 2 * i < ntok ? p0 : 0.f;
+          p1 = 2 * i + 1 < ntok ? p1 : 0.f;
+        }
+        w[i] = M::pack(p0, p1);
+        fadd2(ls[i & 3], M::unpack(w[i]));
+      }
+      const float lsum = (ls[0].x + ls[1].x) + (ls[2].x + ls[3].x) + ((ls[0].y + ls[1].y) + (ls[2].y + ls[3].y));
       // P buffer t % 2 was last read by PV(t-2)
       if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(pv_done(g, sb), ((t - 2) >> 1) & 1, abort_flag))) {
         ok = false;
@@ -400,7 +435,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         tc::tmem_wait_st();
       }
       m = mn;
-      l = l * f + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+      l = l * f + lsum;
       unsigned char* prow_ptr = p_tiles + sb * kPBytes + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
