@@ -168,6 +168,19 @@ def cpu_threads():
         return 1
 
 
+def cpu_model():
+    """Model name of the host CPU (from /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def oracle_sample(sc, seqs, q_host):
     """Time the oracle on sequences ``seqs`` of the scenario's batch; returns (seconds, kv bytes)."""
     from oracle import oracle_decode
@@ -223,7 +236,7 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(sc, args),
             "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host_cpus": os.cpu_count(), "cpu_model": cpu_model()},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -452,7 +465,7 @@ def run_ours(args):
         cpu = {"value": round(nb / dt / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": "%d of %d sequences of one step (%d tokens), float64 numpy, %.1f s" % (
                    len(seqs), sc.batch, sum(int(c.lens[sc.rows.start + s]) for s in seqs), dt),
-               "host_cpus": os.cpu_count()}
+               "host_cpus": os.cpu_count(), "cpu_model": cpu_model()}
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
