@@ -1,5 +1,5 @@
 // sm_100a primitives used by the kernels: shared-memory mbarriers, TMA tile
-// loads and bulk copies (no cluster multicast anywhere), a packed float32x2
+// loads and bulk copies (each CTA loads its own tiles), a packed float32x2
 // FMA, the base-2 exponential instruction, and bounded waits.
 //
 // Every wait is bounded in time: a wait that gives up sets the device error
