@@ -288,17 +288,24 @@ class ReferenceScenario:
         return workloads.queries(self.w, seed, num_seqs=self.batch), None, None
 
 
-def workload_config(sc, args):
+def workload_config(sc, args, l2_bytes=None):
+    """Workload description for the JSON line; ``l2_bytes`` is the device's L2 size (None on the host)."""
     w = sc.w
     lens = sc.cache.lens[sc.rows.start:sc.rows.stop]
+    kv = int(np.sum(lens)) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+    l2 = l2_bytes or 126 * 2**20
+    l2_src = "L2 %d MB from the device" % (l2 // 2**20) if l2_bytes else "L2 126 MB nominal"
+    if kv >= 2 * l2:
+        l2_note = "inputs larger than L2 (K/V set %.2f GB, %s), no flush" % (kv / 1e9, l2_src)
+    else:
+        l2_note = "K/V set %.3f GB under 2x L2 (%s): steps reuse L2, no flush" % (kv / 1e9, l2_src)
     p = w.partition_size if args.partition is None else args.partition
     return {"workload": w.name, "num_seqs": int(sc.batch), "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "block_size": w.block_size, "cache_dtype": w.dtype,
             "mean_context": round(float(np.mean(lens)), 1), "max_context": int(np.max(lens)),
             "partition_size": p, "num_blocks": w.num_blocks, "layers": 1,
             "slot_waste": round(sc.slot_waste(), 5) if hasattr(sc, "slot_waste") else None,
-            "l2": "inputs larger than L2 (K/V set %.2f GB vs 126 MB L2), no flush" % (
-                int(np.sum(lens)) * 2 * w.num_kv_heads * w.head_dim * w.elem_bytes / 1e9),
+            "l2": l2_note,
             "parallelism": "replicas x%d (weak)" % args.gpus}
 
 
@@ -330,7 +337,7 @@ def run_ours(args):
     out = torch.empty((sc.batch, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device="cuda")
     ws = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, part)
     kv_bytes = sc.kv_bytes()
-    config = workload_config(sc, args)
+    config = workload_config(sc, args, torch.cuda.get_device_properties(local).L2_cache_size)
     # copy (when pairs) + append + planner + decode (+ merge with partitions)
     launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 1 + 1 + (1 if part > 0 else 0)
     cascade = args.cascade and w.shared_prefix > 0
