@@ -24,12 +24,14 @@
 //              each softmax group has the other group's products to hide
 //              behind, and tracks completion with tcgen05.commit.
 //   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1; one query
-//              row per thread (tensor-memory lane): load S, online max with
-//              the decode kernel's threshold rule (rescale only when a score
-//              passes the reference by 2^8; O is then rescaled in tensor
-//              memory), P = 2^(s*scale*log2(e) - m) rounded to the cache's
-//              16-bit type and stored back into tensor memory over S as the
-//              A operand of the next product; l sums the rounded weights.
+//              row per thread (tensor-memory lane): one pass over S in
+//              32-column chunks (the next chunk's load in flight), online max
+//              with the decode kernel's threshold rule chunk by chunk (the
+//              reference moves only when a score passes it by 2^8; O and the
+//              tile's stored P chunks are then rescaled in tensor memory),
+//              P = 2^(s*scale*log2(e) - m) rounded to the cache's 16-bit type
+//              and stored back into tensor memory over S as the A operand of
+//              the next product; l sums the rounded weights.
 // Products issued by one thread run in issue order, and a commit arrives only
 // once everything issued before it has completed.  So S(t+1) may overwrite
 // P(t) as soon as PV(t) is issued, and when S(t) is reported ready, PV(t-1)
@@ -363,87 +365,95 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         break;
       }
       tc::fence_after_sync();
-      // Pass 1 over S (64 columns at a time): the row maximum on raw scores;
-      // the scaled maximum is max(s) * qk for qk >= 0 and min(s) * qk
-      // otherwise (rounding is monotonic, so this equals the maximum of the
-      // rounded products).  Columns past a short last tile never win.
+      // One pass over S in 32-column chunks, the load of chunk i + 1 in
+      // flight while chunk i is turned into P.  The reference maximum m
+      // follows the threshold rule chunk by chunk: it moves only when a
+      // chunk's scaled maximum passes it by more than 2^8 (the scaled
+      // maximum is max(s) * qk for qk >= 0 and min(s) * qk otherwise;
+      // rounding is monotonic).  When it moves, O (earlier tiles) and the P
+      // chunks of this tile already stored are rescaled.  P = 2^(s*qk - m) is
+      // rounded to T and packed two per column over scores already read;
+      // lt sums this tile's rounded weights.
       const bool full = ntok == kUmmaTile;
-      float cm[8];
+      float lt = 0.f;
+      uint32_t sbuf[2][32];
+      tc::tmem_ld32(t_lane, sbuf[0]);
+      tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cm[i] = pad;
+      for (int cb = 0; cb < kUmmaTile / 32; ++cb) {
+        uint32_t (&cur)[32] = sbuf[cb & 1];
+        if (cb + 1 < kUmmaTile / 32) tc::tmem_ld32(t_lane + (cb + 1) * 32, sbuf[(cb + 1) & 1]);
+        float cm[4];
 #pragma unroll
-      for (int hb = 0; hb < kUmmaTile / 64; ++hb) {
-        uint32_t sr[2][32];
-        tc::tmem_ld32(t_lane + hb * 64, sr[0]);
-        tc::tmem_ld32(t_lane + hb * 64 + 32, sr[1]);
-        tc::tmem_wait_ld();
+        for (int i = 0; i < 4; ++i) cm[i] = pad;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          float v = __uint_as_float(sr[j >> 5][j & 31]);
-          if (!full) v = hb * 64 + j < ntok ? v : pad;
-          cm[j & 7] = qk >= 0.f ? fmaxf(cm[j & 7], v) : fminf(cm[j & 7], v);
+        for (int j = 0; j < 32; ++j) {
+          float v = __uint_as_float(cur[j]);
+          if (!full) v = cb * 32 + j < ntok ? v : pad;
+          cm[j & 3] = qk >= 0.f ? fmaxf(cm[j & 3], v) : fminf(cm[j & 3], v);
         }
-      }
-      if (qk >= 0.f) {
+        const float ext = qk >= 0.f ? fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]))
+                                    : fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
+        const float c = ext * qk;
+        if (__any_sync(0xffffffffu, c > m + kTau)) {
+          const float mn = c > m + kTau ? c : m;
+          const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
+          if (t >= 1) {
+            // earlier tiles' O: PV(t-1) has completed (S(t) was issued after
+            // it) and PV(t) waits for this tile's P
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cm[i] = fmaxf(cm[i], cm[i + 4]);
-        cm[0] = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
-      } else {
+            for (int ob = 0; ob < D / 32; ++ob) {
+              uint32_t o[32];
+              tc::tmem_ld32(t_lane + 128 + ob * 32, o);
+              tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cm[i] = fminf(cm[i], cm[i + 4]);
-        cm[0] = fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
-      }
-      const float c = cm[0] * qk;
-      const float mn = c > m + kTau ? c : m;
-      float f = 1.f;
-      if (t >= 1 && __any_sync(0xffffffffu, mn != m)) {
-        // the reference maximum moved: PV(t-1) has completed (S(t) was issued
-        // after it) and PV(t) waits for this tile's P, so O may be rescaled
-        f = mn != m ? exp2_approx(m - mn) : 1.f;
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+              tc::tmem_st32(t_lane + 128 + ob * 32, o);
+            }
+          }
+          if (cb > 0) {
+            // this tile's P chunks stored so far, re-rounded; their sum again
+            tc::tmem_wait_st();
+            lt = 0.f;
+            for (int pb = 0; pb < cb; ++pb) {
+              uint32_t pw[16];
+              tc::tmem_ld16(t_lane + pb * 16, pw);
+              tc::tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t o[32];
-          tc::tmem_ld32(t_lane + 128 + cb * 32, o);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-          tc::tmem_st32(t_lane + 128 + cb * 32, o);
+              for (int i = 0; i < 16; ++i) {
+                const float2 u = M::unpack(pw[i]);
+                pw[i] = M::pack(u.x * f, u.y * f);
+                const float2 r = M::unpack(pw[i]);
+                lt += r.x + r.y;
+              }
+              tc::tmem_st16(t_lane + pb * 16, pw);
+            }
+          }
+          l *= f;
+          m = mn;
         }
-      }
-      // Pass 2 (64 columns at a time): P = 2^(s*qk - m) with one packed FMA
-      // per pair, rounded to T and packed two per column; half hb lands in
-      // columns 32hb..32hb+31, which hold scores already read.  The row sum
-      // of the rounded weights uses packed adds.
-      const float2 nm2 = make_float2(-mn, -mn);
-      float2 ls[4];
+        const float2 nm2 = make_float2(-m, -m);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t w[16];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ls[k] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int hb = 0; hb < kUmmaTile / 64; ++hb) {
-        uint32_t sr[2][32];
-        tc::tmem_ld32(t_lane + hb * 64, sr[0]);
-        tc::tmem_ld32(t_lane + hb * 64 + 32, sr[1]);
-        tc::tmem_wait_ld();
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = hb * 64 + 2 * i;
+        for (int i = 0; i < 16; ++i) {
+          const int j = cb * 32 + 2 * i;
           float2 e = nm2;
-          ffma2(e, make_float2(__uint_as_float(sr[i >> 4][(2 * i) & 31]), __uint_as_float(sr[i >> 4][(2 * i + 1) & 31])),
-                qk2);
+          ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
           float p0 = exp2_approx(e.x), p1 = exp2_approx(e.y);
           if (!full) {
             p0 = j < ntok ? p0 : 0.f;
             p1 = j + 1 < ntok ? p1 : 0.f;
           }
           w[i] = M::pack(p0, p1);
-          fadd2(ls[i & 3], M::unpack(w[i]));
+          fadd2(ls[i & 1], M::unpack(w[i]));
         }
-        tc::tmem_st32(t_lane + hb * 32, w);
+        lt += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
+        tc::tmem_st16(t_lane + cb * 16, w);
+        if (cb + 1 < kUmmaTile / 32) tc::tmem_wait_ld();
       }
       tc::tmem_wait_st();
-      m = mn;
-      l = l * f + ((ls[0].x + ls[1].x) + (ls[2].x + ls[3].x) + ((ls[0].y + ls[1].y) + (ls[2].y + ls[3].y)));
+      l += lt;
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full(g));
