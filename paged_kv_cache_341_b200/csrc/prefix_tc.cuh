@@ -383,17 +383,25 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       for (int cb = 0; cb < kUmmaTile / 32; ++cb) {
         uint32_t (&cur)[32] = sbuf[cb & 1];
         if (cb + 1 < kUmmaTile / 32) tc::tmem_ld32(t_lane + (cb + 1) * 32, sbuf[(cb + 1) & 1]);
+        // the sign of qk and whether the tile is full are the same for the
+        // whole warp: one tight loop per case
+        if (!full) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) cur[j] = cb * 32 + j < ntok ? cur[j] : __float_as_uint(pad);
+        }
         float cm[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cm[i] = pad;
+        for (int i = 0; i < 4; ++i) cm[i] = __uint_as_float(cur[i]);
+        float ext;
+        if (qk >= 0.f) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float v = __uint_as_float(cur[j]);
-          if (!full) v = cb * 32 + j < ntok ? v : pad;
-          cm[j & 3] = qk >= 0.f ? fmaxf(cm[j & 3], v) : fminf(cm[j & 3], v);
+          for (int j = 4; j < 32; ++j) cm[j & 3] = fmaxf(cm[j & 3], __uint_as_float(cur[j]));
+          ext = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+        } else {
+#pragma unroll
+          for (int j = 4; j < 32; ++j) cm[j & 3] = fminf(cm[j & 3], __uint_as_float(cur[j]));
+          ext = fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
         }
-        const float ext = qk >= 0.f ? fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]))
-                                    : fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
         const float c = ext * qk;
         if (__any_sync(0xffffffffu, c > m + kTau)) {
           const float mn = c > m + kTau ? c : m;
@@ -435,18 +443,25 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         const float2 nm2 = make_float2(-m, -m);
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         uint32_t w[16];
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = cb * 32 + 2 * i;
-          float2 e = nm2;
-          ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
-          float p0 = exp2_approx(e.x), p1 = exp2_approx(e.y);
-          if (!full) {
-            p0 = j < ntok ? p0 : 0.f;
-            p1 = j + 1 < ntok ? p1 : 0.f;
+          for (int i = 0; i < 16; ++i) {
+            float2 e = nm2;
+            ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
+            w[i] = M::pack(exp2_approx(e.x), exp2_approx(e.y));
+            fadd2(ls[i & 1], M::unpack(w[i]));
           }
-          w[i] = M::pack(p0, p1);
-          fadd2(ls[i & 1], M::unpack(w[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = cb * 32 + 2 * i;
+            float2 e = nm2;
+            ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
+            const float p0 = j < ntok ? exp2_approx(e.x) : 0.f;
+            const float p1 = j + 1 < ntok ? exp2_approx(e.y) : 0.f;
+            w[i] = M::pack(p0, p1);
+            fadd2(ls[i & 1], M::unpack(w[i]));
+          }
         }
         lt += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
         tc::tmem_st16(t_lane + cb * 16, w);
