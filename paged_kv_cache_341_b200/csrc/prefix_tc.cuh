@@ -52,6 +52,18 @@
 
 namespace pa {
 
+// max / min of three float32 values (one instruction on sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // d += a on a pair of float32 lanes (one instruction on sm_100a).
 __device__ __forceinline__ void fadd2(float2& d, const float2 a) {
   asm("{\n\t.reg .b64 rd, ra;\n\t"
@@ -389,18 +401,27 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) cur[j] = cb * 32 + j < ntok ? cur[j] : __float_as_uint(pad);
         }
+        // four chains of three-input max (min) over the 32 scores
         float cm[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) cm[i] = __uint_as_float(cur[i]);
         float ext;
         if (qk >= 0.f) {
 #pragma unroll
-          for (int j = 4; j < 32; ++j) cm[j & 3] = fmaxf(cm[j & 3], __uint_as_float(cur[j]));
-          ext = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+          for (int j = 4; j < 28; j += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cm[k] = fmax3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __uint_as_float(cur[28 + k]));
+          ext = fmax3(fmaxf(cm[0], cm[1]), cm[2], cm[3]);
         } else {
 #pragma unroll
-          for (int j = 4; j < 32; ++j) cm[j & 3] = fminf(cm[j & 3], __uint_as_float(cur[j]));
-          ext = fminf(fminf(cm[0], cm[1]), fminf(cm[2], cm[3]));
+          for (int j = 4; j < 28; j += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cm[k] = fmin3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) cm[k] = fminf(cm[k], __uint_as_float(cur[28 + k]));
+          ext = fmin3(fminf(cm[0], cm[1]), cm[2], cm[3]);
         }
         const float c = ext * qk;
         if (__any_sync(0xffffffffu, c > m + kTau)) {
