@@ -37,6 +37,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; decode tokens/s"
+MIN_ATT_CALLS = 50        # attention calls timed one by one for the roofline (median)
+MAX_ATT_CALLS = 1024
 
 
 def parse():
@@ -381,8 +383,13 @@ def run_ours(args):
         sampler.start()
         time.sleep(0.3)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_att = min(args.steps, 256)
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_att)]
+    # the attention call of each step is bracketed by events (median reported);
+    # with fewer than MIN_ATT_CALLS steps, further steps after the timed region
+    # (same step, same inputs, still under the clock sampler) supply the rest
+    n_att = min(args.steps, MAX_ATT_CALLS)
+    n_extra = max(0, MIN_ATT_CALLS - n_att)
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_att + n_extra)]
     t_start.record(stream)
     for i in range(args.steps):
         if i < n_att:
@@ -390,12 +397,15 @@ def run_ours(args):
         else:
             step()
     t_end.record(stream)
+    for i in range(n_extra):
+        step(*att_ev[n_att + i])
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
     ms = t_start.elapsed_time(t_end) / args.steps
-    att_ms = float(np.mean([a.elapsed_time(b) for a, b in att_ev]))
+    att_times = [a.elapsed_time(b) for a, b in att_ev]
+    att_ms = float(np.median(att_times))
     ms, att_ms = max_over_ranks([ms, att_ms], device="cuda")
     assert pa.pa_device_error() == 0
 
@@ -489,11 +499,16 @@ def run_ours(args):
             "decode_tokens_per_s": round(world * sc.batch / (ms / 1e3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": "pa_decode_attention call (%s + reduce_kernel), mean of %d calls; "
-                                   "peak = %s copy bandwidth" % (
+                         "kernel": "pa_decode_attention call (plan_kernel + %s + reduce_kernel), median of %d "
+                                   "calls; peak = %s copy bandwidth" % (
                                        "decode_mma_kernel" if w.elem_bytes == 2 and
                                        os.environ.get("PA_DECODE_PATH") != "alu" else "decode_kernel",
-                                       n_att, peak_kind),
+                                       len(att_times), peak_kind),
+                         "timed_calls": len(att_times),
+                         "statistic": "median",
+                         "call_ms": {"median": round(float(np.median(att_times)), 5),
+                                     "p10": round(float(np.percentile(att_times, 10)), 5),
+                                     "p90": round(float(np.percentile(att_times, 90)), 5)},
                          "algorithmic_bytes_per_launch": kv_bytes,
                          "read_ceiling": {"value": round(read_gbs, 2), "unit": "GB/s",
                                           "kernel": "read_stream_kernel (pa_read_stream): %.2f GB buffer read once "

@@ -304,14 +304,20 @@ pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, 
  * Arguments and results are those of pa_decode_attention without
  * `workspace`/`workspace_bytes`.  PA_ERR_INVALID, with a message naming the
  * size, when pa_decode_workspace_size(...) for these sizes exceeds
- * PA_STATIC_WORKSPACE_BYTES (partition_size == 0 needs none).
+ * PA_STATIC_WORKSPACE_BYTES.  That limit applies to partition_size == 0 as
+ * well: the single-pass path keeps its work list in the array too (256 bytes
+ * plus 16 bytes per sequence and query head).
  *
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  All calls
- * on a device share the one array, which keeps whatever the last call left in
- * it (nothing in it has to start at zero: every partial is written before it
- * is read within a call).  Calls that overlap on the GPU -- on different
- * streams, or from different host threads -- race on it; serialise them. */
+ * Every call looks up the array's device address in the current device's
+ * context (cudaGetSymbolAddress; no allocation).  The first call in a context
+ * also loads the library's device code there, so make that first call on a
+ * device before any stream capture.  All calls on a device share the one
+ * array, which keeps whatever the last call left in it (nothing in it has to
+ * start at zero: the work counter is reset and every partial is written
+ * before it is read within a call).  Calls issued one after another on one
+ * stream are ordered on the array.  Calls that overlap on the GPU -- on
+ * different streams, or from different host threads -- race on it; serialise
+ * them. */
 pa_status pa_decode_attention_static(const void* q, const void* k_cache, const void* v_cache,
                                      int32_t num_blocks, const int32_t* block_tables,
                                      int32_t max_blocks_per_seq, const int32_t* context_lens,
@@ -400,8 +406,23 @@ pa_status pa_engine_synchronize(pa_engine* engine);
 /* Read (and, if reset != 0, clear) the device error word of the current
  * device: 0 = none; 1 = block id outside the pool in a table; 2 =
  * context length beyond the table; 3 = append slot outside the cache; 4 =
- * copy pair id outside the pool.  Synchronous: waits for the device. */
+ * copy pair id outside the pool; 5 = a pipeline wait of a kernel ran out of
+ * time (that kernel returned early and its output is undefined).
+ * Synchronous: waits for the device. */
 pa_status pa_device_error(int32_t* code_out, int32_t reset);
+
+/* Test hook for the bounded waits of the decode kernel; not a step of the
+ * path, and off unless a test turns it on.  Every wait inside the kernels is
+ * bounded in time: a wait that runs out sets device error 5, tells the other
+ * warps of its CTA to stop, lets the copies already in flight land, and
+ * returns, so a lost arrival can never hang the GPU.  With wait_limit_ns > 0
+ * (between 1e3 and 2e9) every following pa_decode_attention launch (until
+ * the hook is turned off with 0) uses that bound instead of the normal 2 s,
+ * and the producer warp of every decode CTA withholds its first pipeline
+ * stage, so the consumer's wait for it is certain to run out: the call
+ * completes, its output is undefined, and pa_device_error reports 5.
+ * Process-wide setting; PA_ERR_INVALID for a bound outside the range. */
+pa_status pa_debug_decode_stall(int64_t wait_limit_ns);
 
 /* Message of the last failing call on this thread ("" if none). */
 const char* pa_last_error(void);

@@ -88,6 +88,8 @@ struct DecodeParams {
   uint32_t tile_bytes;           // bytes of one K (or V) stage tile
   uint32_t q_bytes;              // bytes of one unit's query rows
   float qk_scale;                // scale * log2(e)
+  uint64_t wait_limit_ns;        // bound of every pipeline wait (kWaitLimitNs unless a test shortens it)
+  int withhold_first;            // test hook, 0 in every normal call: see pa_debug_decode_stall
 };
 
 struct StageMeta {
@@ -221,7 +223,9 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
   bool ok = true;
 
   // Planned order: claim the next unit index and fetch its descriptor one
-  // unit ahead (lane 0), so both round trips overlap the current unit.
+  // unit ahead (lane 0), so both round trips overlap the current unit.  The
+  // plan lists (sequence, partition) entries; unit c is KV-head tile c % n_tiles
+  // of entry c / n_tiles, so the tiles of one partition are taken together.
   const bool planned = prm.units != nullptr;
   int total_units = 0;
   int4 next_desc = make_int4(-1, 0, 0, 0);
@@ -229,7 +233,11 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
     int4 d = make_int4(-1, 0, 0, 0);
     if (lane == 0) {
       const int c = atomicAdd(prm.sched, 1);
-      if (c < total_units) d = __ldcg(prm.units + c);
+      if (c < total_units) {
+        const int e = c / n_tiles;
+        d = __ldcg(prm.units + e);
+        d.z = c - e * n_tiles;
+      }
     }
     return d;
   };
@@ -291,7 +299,8 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
     const int qslot = units_done & 1;
 
     // Query rows of this unit: [HT*G][D] contiguous in q.
-    if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_empty[qslot], ((units_done >> 1) & 1) ^ 1, pl.abort_flag))) {
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&pl.q_empty[qslot], ((units_done >> 1) & 1) ^ 1, pl.abort_flag, prm.wait_limit_ns))) {
       ok = false;
       break;
     }
@@ -333,11 +342,14 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
         rows[pc] = phys * BS + within;
         loaded = pc + 1;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag, prm.wait_limit_ns))) {
         ok = false;
         break;
       }
-      if (lane == 0) {
+      // test hook: the first arming of the CTA is never made, so the consumers'
+      // wait for it runs out (never set in a normal call)
+      const bool withhold = prm.withhold_first && armed == 0;
+      if (lane == 0 && !withhold) {
         StageMeta m;
         m.seq = seq;
         m.part = part;
@@ -355,7 +367,7 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
         }
       }
       __syncwarp();
-      if (loaded > 0) {
+      if (loaded > 0 && !withhold) {
         T* dk = pl.s_k + stage * pl.tile_elems;
         T* dv = pl.s_v + stage * pl.tile_elems;
         if constexpr (kSwizzled) {
@@ -389,8 +401,8 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
 
   if (ok) {
     // End-of-work marker for the consumers.
-    if (__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag))) {
-      if (lane == 0) {
+    if (__all_sync(0xffffffffu, mbar_wait(&pl.empty[stage], phase ^ 1, pl.abort_flag, prm.wait_limit_ns))) {
+      if (lane == 0 && !(prm.withhold_first && armed == 0)) {
         pl.meta[stage].seq = -1;
         mbar_arrive(&pl.full[stage]);
       }
@@ -413,11 +425,11 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
         st = stages - 1;
         ph ^= 1;
       }
-      mbar_wait_drain(&pl.full[st], ph);
+      mbar_wait_drain(&pl.full[st], ph, prm.wait_limit_ns);
     }
     for (int k = 1; k <= 2 && k <= q_issued; ++k) {
       const int un = q_issued - k;
-      mbar_wait_drain(&pl.q_full[un & 1], (un >> 1) & 1);
+      mbar_wait_drain(&pl.q_full[un & 1], (un >> 1) & 1, prm.wait_limit_ns);
     }
   }
   __syncwarp();
@@ -475,12 +487,14 @@ __global__ void __launch_bounds__((kMaxTileHeads + 1) * 32, 1)
   int units_done = 0;
 
   while (true) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag))) return;
+    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag, prm.wait_limit_ns))) return;
     const StageMeta mt = pl.meta[stage];
     if (mt.seq < 0) return;
 
     if (mt.flags & kFirst) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag))) return;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag, prm.wait_limit_ns)))
+        return;
       const T* qrow = pl.s_q + mt.qslot * HT * G * D + j * G * D;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -745,12 +759,14 @@ __global__ void __maxnreg__(128)
   int units_done = 0;
 
   while (true) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag))) return;
+    if (!__all_sync(0xffffffffu, mbar_wait(&pl.full[stage], phase, pl.abort_flag, prm.wait_limit_ns))) return;
     const StageMeta mt = pl.meta[stage];
     if (mt.seq < 0) return;
 
     if (mt.flags & kFirst) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag))) return;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&pl.q_full[mt.qslot], (units_done >> 1) & 1, pl.abort_flag, prm.wait_limit_ns)))
+        return;
       const T* qbase = pl.s_q + mt.qslot * HT * G * D + j * G * D;
 #pragma unroll
       for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -902,21 +918,26 @@ __global__ void __maxnreg__(128)
 }
 
 // ===========================================================================
-// Planner: the decode kernel's unit list.  Full partitions first, in
-// sequence order with the KV-head tiles of a partition next to each other
-// (they read the same blocks); then the remainder partitions -- or, without
-// partitions, the whole sequences -- by decreasing length (counting sort on
-// 16-token chunks), so the smallest units are taken last.  One CTA; also
-// zeroes the unit counter and stores the unit count.  It is launched as a
-// programmatic dependent of the kernel before it (the append of the step) and
-// reads only the lengths, so it overlaps that kernel; before exiting it waits
-// for it, so a decode grid that has waited for the planner also sees the
-// appended K/V.
+// Planner: the decode kernel's work list, one entry {seq, part, -, len} per
+// (sequence, partition); the decode grid expands each entry into its
+// n_tiles KV-head tiles, taken one after another (they read the same
+// blocks).  Full partitions first, in sequence order; then the remainder
+// partitions -- or, without partitions, the whole sequences -- by decreasing
+// length (counting sort on 16-token chunks), so the smallest units are taken
+// last.  One CTA; also zeroes the unit counter and stores the unit count.
+//
+// It is launched as a programmatic dependent of the kernel before it on the
+// stream and lets the decode grid launch at once (its CTAs set up and then
+// wait for the planner), but it reads and writes nothing before its own
+// griddepcontrol.wait has returned.  That wait matters twice over: the kernel
+// before may be the previous call's decode grid, still claiming units from
+// the same workspace (resetting the counter under it would hand it this
+// call's units), or it may be the kernel that wrote the lengths.
 // ===========================================================================
 struct PlanParams {
   const int32_t* context_lens;
-  int4* units;                   // {seq, part, tile, len}
-  int* header;                   // [0] unit counter (zeroed), [1] unit count
+  int4* units;                   // entries {seq, part, 0, len}, one per (sequence, partition)
+  int* header;                   // [0] unit counter (zeroed), [1] unit count (entries x num_tiles)
   int num_seqs, partition_size, num_tiles, cap;
 };
 
@@ -954,7 +975,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm) {
   __shared__ int bucket[kPlanBuckets];
   __shared__ int warp_sums[32];
-  allow_dependent_launch();                    // the decode grid may start; it waits for this one
+  allow_dependent_launch();                    // the decode grid may launch; it waits for this one
+  wait_prerequisite_grids();                   // the kernel before has finished and its writes are visible
   const int tid = threadIdx.x;
   const int S = prm.num_seqs, P = prm.partition_size, nt = prm.num_tiles;
   for (int b = tid; b < kPlanBuckets; b += kPlanThreads) bucket[b] = 0;
@@ -986,12 +1008,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
       if (b >= 0) atomicAdd(&bucket[b], 1);
     }
     int round_total;
-    const int off = block_exclusive_scan(nfull * nt, warp_sums, &round_total);
-    for (int p = 0; p < nfull; ++p)
-      for (int t = 0; t < nt; ++t) prm.units[written + off + p * nt + t] = make_int4(s, p, t, len);
+    const int off = block_exclusive_scan(nfull, warp_sums, &round_total);
+    for (int p = 0; p < nfull; ++p) prm.units[written + off + p] = make_int4(s, p, 0, len);
     written += round_total;
   }
-  // bucket starts, largest remainders first: start[b] = written + nt * sum_{b' > b} count[b']
+  // bucket starts, largest remainders first: start[b] = written + sum_{b' > b} count[b']
   {
     constexpr int PER = kPlanBuckets / kPlanThreads;
     int local[PER];
@@ -1008,13 +1029,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
     for (int i = 0; i < PER; ++i) {
       const int b = kPlanBuckets - 1 - (tid * PER + i);
       const int c = local[i];
-      bucket[b] = written + run * nt;             // becomes the cursor of bucket b
+      bucket[b] = written + run;                  // becomes the cursor of bucket b
       run += c;
     }
     __syncthreads();
     if (tid == 0) {
       prm.header[0] = 0;
-      prm.header[1] = written + tot * nt;
+      prm.header[1] = (written + tot) * nt;
     }
   }
   // pass 1: remainder partitions into their buckets
@@ -1022,11 +1043,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
     const int len = load_len(s);
     const int b = rem_bucket(len);
     if (b < 0) continue;
-    const int pos = atomicAdd(&bucket[b], nt);
+    const int pos = atomicAdd(&bucket[b], 1);
     const int part = P > 0 ? len / P : 0;
-    for (int t = 0; t < nt; ++t) prm.units[pos + t] = make_int4(s, part, t, len);
+    prm.units[pos] = make_int4(s, part, 0, len);
   }
-  wait_prerequisite_grids();
 }
 
 // ===========================================================================
@@ -1053,10 +1073,10 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   constexpr int PER = D / 32;                // contiguous elements per lane
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
   const int s = blockIdx.y;
-  int len = prm.context_lens[s];             // written before the decode launch: safe to read now
+  wait_prerequisite_grids();                 // the decode grid (and all before it) is done and visible
+  int len = prm.context_lens[s];
   len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
   const int np = prm.part_offset + parts_of(len, prm.partition_size);
-  wait_prerequisite_grids();
   if (prm.part_offset == 0 && np <= 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hq = blockIdx.x * kReduceWarps + warp;

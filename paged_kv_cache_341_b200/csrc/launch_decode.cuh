@@ -10,6 +10,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
@@ -67,6 +68,11 @@ pa_status device_info(DeviceInfo* out) {
   *out = d;
   return PA_OK;
 }
+
+// Test hook of pa_debug_decode_stall: 0 = off (every normal call); otherwise
+// the wait bound in nanoseconds, and every decode CTA withholds its first
+// stage so that its consumers' bounded wait runs out.
+std::atomic<long long> g_decode_stall_ns{0};
 
 // Optional tuning overrides (no effect on results): KV heads per CTA tile and
 // pipeline depth of the decode kernel.
@@ -247,6 +253,9 @@ pa_status launch_decode(const DecodeArgs& a) {
   prm.tile_bytes = static_cast<uint32_t>(tile_bytes);
   prm.q_bytes = static_cast<uint32_t>(q_bytes);
   prm.qk_scale = a.scale * 1.4426950408889634f;
+  const long long stall_ns = g_decode_stall_ns.load(std::memory_order_relaxed);
+  prm.wait_limit_ns = stall_ns > 0 ? static_cast<uint64_t>(stall_ns) : pa::kWaitLimitNs;
+  prm.withhold_first = stall_ns > 0 ? 1 : 0;
 
   if (prm.units) {
     // planner (one CTA), then the decode grid as its programmatic dependent

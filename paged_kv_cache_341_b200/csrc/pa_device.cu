@@ -327,23 +327,17 @@ static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORK
 
 namespace {
 
-// Device address of g_static_workspace on the current device, looked up once
-// per device (the host-side symbol is only a stand-in, not a device address).
+// Device address of g_static_workspace in the current device's context.  In
+// host code the symbol is only a stand-in, not a device address, and the
+// address belongs to a context (it changes after cudaDeviceReset, and differs
+// under another driver context), so it is looked up on every call rather than
+// cached: the lookup allocates nothing.  The first lookup in a context loads
+// the library's device code into it.
 pa_status static_workspace(void** out) {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode_attention_static: device index >= 64");
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_workspace);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+  *out = p;
   return PA_OK;
 }
 
@@ -435,6 +429,13 @@ pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, 
   if (st != PA_OK) return st;
   st = dtype == PA_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
   return st == PA_OK ? pa::ok() : st;
+}
+
+pa_status pa_debug_decode_stall(int64_t wait_limit_ns) {
+  if (wait_limit_ns != 0 && (wait_limit_ns < 1000 || wait_limit_ns > static_cast<int64_t>(pa::kWaitLimitNs)))
+    return pa::fail(PA_ERR_INVALID, "pa_debug_decode_stall: wait_limit_ns must be 0 or in [1e3, 2e9]");
+  g_decode_stall_ns.store(wait_limit_ns, std::memory_order_relaxed);
+  return pa::ok();
 }
 
 pa_status pa_device_error(int32_t* code_out, int32_t reset) {

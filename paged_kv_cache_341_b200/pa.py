@@ -63,6 +63,7 @@ SIGNATURES = {
     "pa_decode_attention_shared_prefix": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _vp, _i32, _i32,
                                                  _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _i32, _vp]),
     "pa_device_error": (_i32, [_p32, _i32]),
+    "pa_debug_decode_stall": (_i32, [_i64]),
     "pa_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -377,6 +378,11 @@ def pa_device_error(reset=True):
     code = ctypes.c_int32()
     _check(_lib.pa_device_error(ctypes.byref(code), 1 if reset else 0))
     return code.value
+
+
+def pa_debug_decode_stall(wait_limit_ns):
+    """Test hook of the bounded waits (0 = off): see include/pa.h."""
+    _check(_lib.pa_debug_decode_stall(int(wait_limit_ns)))
 
 
 # --------------------------------------------------------------------------

@@ -58,3 +58,27 @@ def build_pool_contents(pool_shape, dtype, tables, lens, block_size, seed, poiso
                 k[last, n % block_size:] = float("nan")
                 v[last, n % block_size:] = float("nan")
     return k, v
+
+
+def full_table_case(num_seqs, max_blocks, block_size, num_kv_heads, head_dim, dtype, seed):
+    """A cache whose every block-table entry names a valid, filled block.
+
+    Each of ``num_seqs`` rows owns ``max_blocks`` blocks (from a seeded
+    shuffled pool), so any length up to ``max_blocks * block_size`` can be
+    attended without touching an unfilled slot.  Returns (cache, k_host,
+    v_host, host tables as lists)."""
+    from paged_kv_cache_341_b200.cache import PagedKVCache
+    rng = np.random.default_rng(seed)
+    cap = max_blocks * block_size
+    nb = num_seqs * max_blocks + 2
+    cache = PagedKVCache(nb, block_size, num_kv_heads, head_dim, TORCH[dtype], num_seqs, max_blocks,
+                         initial_free_order=rng.permutation(nb))
+    for row in range(num_seqs):
+        cache.allocate(row, cap)
+    full = [cap] * num_seqs
+    k, v = build_pool_contents((nb, block_size, num_kv_heads, head_dim), dtype, cache.tables, full, block_size,
+                               seed + 1)
+    cache.k_cache.copy_(k)
+    cache.v_cache.copy_(v)
+    cache.upload_tables()
+    return cache, k, v, [list(r) for r in cache.tables]

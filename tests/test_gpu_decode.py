@@ -253,3 +253,52 @@ def test_device_checks_flag_bad_indices(pa):
     cache.upload_tables()
     cache.attend(q, out, 0.125)
     assert pa.pa_device_error() == 0
+
+
+@pytest.mark.parametrize("partition", [0, 256])
+def test_bounded_wait_runs_out_and_returns(pa, path, partition):
+    """Every pipeline wait is bounded: with the test hook on, the producer of
+    every decode CTA withholds its first stage, so the consumer's wait for it
+    can only run out.  After 1 ms it does; every warp returns, the copies in
+    flight land, the call completes and the device error word says 5
+    (timeout).  The context stays usable: the next normal call is correct."""
+    from paged_kv_cache_341_b200.cache import PagedKVCache
+    lens = [1, 40, 700, 1500, 16, 0, 333]
+    s, hq, hkv, d, bs = len(lens), 16, 4, 128, 16
+    rng = np.random.default_rng(61)
+    nb = sum(-(-n // bs) for n in lens) + 2
+    mb = max(-(-n // bs) for n in lens) + 1
+    cache = PagedKVCache(nb, bs, hkv, d, torch.bfloat16, s, mb, initial_free_order=rng.permutation(nb))
+    for row, n in enumerate(lens):
+        cache.allocate(row, n)
+    k_host, v_host = build_pool_contents((nb, bs, hkv, d), "bf16", cache.tables, lens, bs, 62)
+    cache.k_cache.copy_(k_host)
+    cache.v_cache.copy_(v_host)
+    cache.upload_tables()
+    q_host = workloads.randn((s, hq, d), "bf16", 63)
+    q = q_host.cuda()
+    scale = 1.0 / math.sqrt(d)
+    ws = pa.decode_workspace(s, hq, d, mb, bs, partition)
+    out = torch.zeros((s, hq, d), dtype=torch.bfloat16, device="cuda")
+    assert pa.pa_device_error(reset=True) == 0
+    pa.pa_debug_decode_stall(1_000_000)
+    try:
+        cache.attend(q, out, scale, partition, ws)
+        code = pa.pa_device_error(reset=True)       # synchronises: the call has completed
+    finally:
+        pa.pa_debug_decode_stall(0)
+    assert code == 5
+    good = torch.full_like(out, float("nan"))
+    cache.attend(q, good, scale, partition, ws)
+    assert pa.pa_device_error() == 0
+    ref = oracle_decode(q_host.double().numpy(), AsF64(k_host), AsF64(v_host), [list(r) for r in cache.tables],
+                        lens, scale)
+    assert_close(good.float().cpu().numpy(), ref, "bf16", "after a timed-out call")
+
+
+def test_stall_hook_rejects_bad_bounds(pa):
+    for bad in (-1, 10, 3_000_000_000):
+        with pytest.raises(pa.PagedAttnError) as e:
+            pa.pa_debug_decode_stall(bad)
+        assert e.value.status == pa.PA_ERR_INVALID
+    pa.pa_debug_decode_stall(0)

@@ -1,9 +1,23 @@
 """Full-size workloads on the GPU, in the launch configuration the benchmark
-times (one decode step: reserve, copy-on-write, append, partitioned attention
-with 512-token partitions), checked against the oracle replaying the same
-steps: block tables, slots, copy pairs and pool state bit-exact, appended
-rows and copied blocks bit-exact, and attention on sampled (sequence, head)
-outputs within tolerance (every output must be finite)."""
+times: one decode step (reserve, copy-on-write, append, partitioned
+attention with the workload's partition size plus the merge), checked
+against the oracle replaying the same steps.
+
+* block tables, slots, copy pairs and pool state: bit-exact;
+* appended rows and copied blocks: bit-exact;
+* attention: every (sequence, query head) output against the oracle for the
+  Llama-2-7B, Llama-3-8B and 70B-shaped workloads; for the shared-prefix
+  workload (200 sequences x 30,720 + suffix tokens, about 100 GFLOP of
+  float64 work for all of them) a stratified sample of sequences covering
+  every 128-row query tile of the prefix kernel, all heads, against the
+  oracle, and every output of the cascade call against the plain call.
+
+The shared-prefix workload is the "Paged Attention" glossary's example (a
+30k-token prompt shared by 200 users; aidolsgroup.com, section "Example") and
+agentechip.com's "Shared Prefix Caching".
+"""
+
+import math
 
 import numpy as np
 import pytest
@@ -43,10 +57,23 @@ def oracle_replay(sc):
     return op, tables, lens
 
 
-@pytest.mark.parametrize("name", ["llama2_7b_mha", "llama3_8b_gqa", "shared_prefix", "long_70b_gqa"])
-def test_full_size_step(name):
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
+def prefix_tile_sample(batch, group, rng, per_tile=4):
+    """Sequences covering every 128-row query tile of one KV head (rows s * group + g):
+    the first and last sequence of each tile and ``per_tile - 2`` others."""
+    seqs_per_tile = 128 // group
+    picks = set()
+    for t0 in range(0, batch, seqs_per_tile):
+        t1 = min(batch, t0 + seqs_per_tile) - 1
+        picks |= {t0, t1}
+        inner = list(range(t0 + 1, t1))
+        if inner:
+            picks |= set(int(x) for x in rng.choice(inner, min(per_tile - 2, len(inner)), replace=False))
+    return sorted(picks)
+
+
+def full_step(name):
+    """Build the workload, take one decode step through the library and the oracle; check the
+    bit-exact parts.  Returns what the attention checks need."""
     from paged_kv_cache_341_b200 import pa
     from paged_kv_cache_341_b200.scenarios import Scenario
     sc = Scenario(name, keep_host=True)
@@ -65,7 +92,8 @@ def test_full_size_step(name):
     q, k_new, v_new = sc.step_inputs(0)
     out = torch.full((sc.batch, w.num_q_heads, w.head_dim), float("nan"), dtype=w.torch_dtype, device="cuda")
     ws = pa.decode_workspace(sc.batch, w.num_q_heads, w.head_dim, c.max_blocks, w.block_size, w.partition_size)
-    slots, pairs = c.decode_step(q.cuda(), k_new.cuda(), v_new.cuda(), out, w.scale, w.partition_size, ws,
+    q_dev = q.cuda()
+    slots, pairs = c.decode_step(q_dev, k_new.cuda(), v_new.cuda(), out, w.scale, w.partition_size, ws,
                                  rows=sc.rows)
     torch.cuda.synchronize()
     assert pa.pa_device_error() == 0
@@ -90,24 +118,60 @@ def test_full_size_step(name):
         assert list(c.d_tables[r, :nblk].cpu().numpy()) == otables[r]
     assert list(c.d_lens.cpu().numpy()) == olens
 
-    # bit-exact: appended rows and copied blocks
+    # bit-exact: appended rows and every copied block
     flat_k = c.k_cache.view(-1, w.num_kv_heads, w.head_dim)
     flat_v = c.v_cache.view(-1, w.num_kv_heads, w.head_dim)
     idx = torch.tensor(oslots, dtype=torch.int64, device="cuda")
     assert torch.equal(flat_k[idx].cpu(), k_new) and torch.equal(flat_v[idx].cpu(), v_new)
-    for src, dst in opairs[:64]:
+    for src, dst in opairs:
         assert torch.equal(c.k_cache[dst].cpu(), sc.k_host[dst]) and torch.equal(c.v_cache[dst].cpu(), sc.v_host[dst])
 
-    # attention: every output finite; sampled outputs against the oracle
-    gpu = out.float().cpu().numpy()
-    assert np.all(np.isfinite(gpu))
-    rng = np.random.default_rng(341)
-    blens = np.array(olens[sc.rows.start:sc.rows.stop])
-    picks = {int(np.argmax(blens)), int(np.argmin(blens))} | set(int(x) for x in rng.choice(sc.batch, min(10, sc.batch), False))
     btables = otables[sc.rows.start:sc.rows.stop]
-    kw, vw = AsF64(sc.k_host), AsF64(sc.v_host)
-    qd = q.double().numpy()
-    for sidx in sorted(picks):
-        heads = sorted(set(int(h) for h in rng.choice(w.num_q_heads, 4, False)) | {0, w.num_q_heads - 1})
-        ref = oracle_decode(qd, kw, vw, btables, blens, w.scale, seqs=[sidx], heads=heads)
-        assert_close(gpu[sidx, heads], ref[sidx, heads], w.dtype, "%s seq %d" % (name, sidx))
+    blens = [int(x) for x in olens[sc.rows.start:sc.rows.stop]]
+    return sc, q, q_dev, out, btables, blens
+
+
+@pytest.mark.parametrize("name", ["llama2_7b_mha", "llama3_8b_gqa", "long_70b_gqa"])
+def test_full_size_step(name):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    sc, q, _, out, btables, blens = full_step(name)
+    w = sc.w
+    ref = oracle_decode(q.double().numpy(), AsF64(sc.k_host), AsF64(sc.v_host), btables, blens, w.scale)
+    assert_close(out.float().cpu().numpy(), ref, w.dtype, "%s, every (sequence, head)" % name)
+
+
+def test_shared_prefix_full_size_step_plain_and_cascade(monkeypatch):
+    """The shared-prefix step: copy-on-write of the forks' partly filled last blocks, append,
+    then attention twice over the same state -- the plain partitioned call and the cascade
+    call (prefix once for all 200 x 32 query rows on the tcgen05 kernel, 30 slices of 1,024
+    tokens, suffix partitions of 512, merge)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_cache_341_b200 import pa
+    sc, q, q_dev, plain, btables, blens = full_step("shared_prefix")
+    w, c = sc.w, sc.cache
+    monkeypatch.setenv("PA_PREFIX_PATH", "umma")
+    pblocks = w.shared_prefix // w.block_size
+    prefix_ids = c.d_tables[sc.rows.start, :pblocks].contiguous()
+    suffix_tables = c.d_tables[sc.rows, pblocks:]
+    suffix_lens = (c.d_lens[sc.rows] - w.shared_prefix).contiguous()
+    ws = torch.empty(pa.pa_shared_prefix_workspace_size(sc.batch, w.num_q_heads, w.head_dim, w.shared_prefix,
+                                                        suffix_tables.shape[1], w.block_size, w.partition_size),
+                     dtype=torch.uint8, device="cuda")
+    casc = torch.full_like(plain, float("nan"))
+    pa.pa_decode_attention_shared_prefix(q_dev, c.k_cache, c.v_cache, prefix_ids, w.shared_prefix, suffix_tables,
+                                         suffix_lens, w.scale, casc, w.partition_size, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+    for r in range(sc.batch):
+        assert btables[r][:pblocks] == btables[0][:pblocks]
+    plain_h = plain.float().cpu().numpy()
+    casc_h = casc.float().cpu().numpy()
+    assert_close(casc_h, plain_h, w.dtype, "cascade vs plain call, all 200 x 32 outputs")
+    group = w.num_q_heads // w.num_kv_heads
+    picks = prefix_tile_sample(sc.batch, group, np.random.default_rng(341))
+    assert len(picks) >= 24 and picks[-1] == sc.batch - 1
+    ref = oracle_decode(q.double().numpy(), AsF64(sc.k_host), AsF64(sc.v_host), btables, blens, w.scale, seqs=picks)
+    assert_close(plain_h[picks], ref[picks], w.dtype, "plain call, %d sampled sequences" % len(picks))
+    assert_close(casc_h[picks], ref[picks], w.dtype, "cascade call, %d sampled sequences" % len(picks))
