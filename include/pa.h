@@ -128,6 +128,19 @@ pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, in
                            int32_t num_seqs, int64_t* slots_out, int32_t* pairs_out,
                            int32_t* num_pairs_out);
 
+/* pa_reserve_slots that also lists the block-table entries the step wrote,
+ * for a caller that keeps a device copy of the tables up to date without
+ * re-sending them: updates_out ([S][3] room, host) receives one
+ * (row0 + s, column, block id) triple for every sequence s whose reserved
+ * token took a block -- a fresh block at offset 0, or the private copy of a
+ * shared block -- and *num_updates_out their count.  These are exactly the
+ * entries to pass to pa_update_block_tables.  updates_out may be NULL (then
+ * this is pa_reserve_slots).  All or nothing, as pa_reserve_slots. */
+pa_status pa_reserve_slots_with_updates(pa_pool* pool, int32_t* tables, int32_t table_cap, int32_t* lens,
+                                        int32_t num_seqs, int32_t row0, int64_t* slots_out,
+                                        int32_t* pairs_out, int32_t* num_pairs_out,
+                                        int32_t* updates_out, int32_t* num_updates_out);
+
 /* Prefix caching by block content ("Paged Attention", aidolsgroup.com, "Why
  * it matters": every KV-cache block is hashed by its tokens and the tokens
  * before it, so requests sharing a system prompt reuse the same blocks).

@@ -98,13 +98,19 @@ def up_to_date():
 
 
 def ensure_built():
-    """Build when the library is missing or its sources changed; returns the path."""
+    """Build when the library is missing, its sources changed, or its build record is missing.
+
+    A library without ``_build/digest.txt`` beside it cannot be tied to the
+    sources in the tree, so it is rebuilt rather than trusted; if that build
+    fails, the error says so instead of loading a library of unknown origin.
+    Returns the path."""
     if up_to_date():
         return LIB
-    if os.path.exists(LIB) and not os.path.exists(os.path.join(BUILD, "digest.txt")):
-        # shipped without build metadata (e.g. copied onto a GPU box): trust it
-        return LIB
-    return build()
+    try:
+        return build()
+    except (OSError, RuntimeError) as e:
+        raise RuntimeError("libpagedattn.so is missing or does not match its sources (no build record, or "
+                           "a different digest), and rebuilding it failed: %s" % e) from e
 
 
 if __name__ == "__main__":

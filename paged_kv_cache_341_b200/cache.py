@@ -169,33 +169,22 @@ class PagedKVCache:
         stream = stream or torch.cuda.current_stream()
         sel = slice(None) if rows is None else rows
         r0 = sel.start or 0
-        lens_view = self.lens[sel]
-        tab_view = self.tables[sel]
-        n = lens_view.size
-        idx = np.arange(n)
-        cols = lens_view // self.block_size
-        old = tab_view[idx, np.minimum(cols, self.max_blocks - 1)].copy()
-        fresh = (lens_view % self.block_size) == 0
-        slots, pairs = self.reserve(rows)
-        new = tab_view[idx, cols]
-        changed = np.nonzero(fresh | (new != old))[0]
+        tables = self.tables[sel]
+        lens = self.lens[sel]
+        assert tables.flags.c_contiguous and lens.flags.c_contiguous
+        n = lens.size
         b = self._step & 1
-        self._step += 1
         if self._meta_done[b] is not None:
             self._meta_done[b].synchronize()          # the H2D out of this host slot has finished
         h_slots, h_lens, h_upd, h_pairs = self._meta_views[b]
         d_slots, d_lens, d_upd, d_pairs = self._meta_dviews[b]
-        h_slots.numpy()[:n] = slots
+        # the reservation writes the slots, pairs and changed table entries straight into the staging
+        npairs, nu = self.pool.pa_reserve_slots_with_updates(tables, lens, r0, h_slots.numpy()[:n],
+                                                             h_pairs.numpy(), h_upd.numpy())
+        self._step += 1
+        slots = h_slots.numpy()[:n].copy()
+        pairs = h_pairs.numpy()[:npairs].copy()
         h_lens.numpy()[:self.lens.size] = self.lens
-        nu = changed.size
-        if nu:
-            u = h_upd.numpy()
-            u[:nu, 0] = changed + r0
-            u[:nu, 1] = cols[changed]
-            u[:nu, 2] = new[changed]
-        npairs = pairs.shape[0]
-        if npairs:
-            h_pairs.numpy()[:npairs] = pairs
         with torch.cuda.stream(stream):
             self._meta_dev[b].copy_(self._meta_host[b], non_blocking=True)
             ev = torch.cuda.Event()

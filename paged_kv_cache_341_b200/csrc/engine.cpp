@@ -76,7 +76,6 @@ struct pa_engine {
   cudaEvent_t out_read[kSlots] = {};
   bool used[kSlots] = {false, false};
   int64_t steps = 0;
-  std::vector<int32_t> old_entry;
 
   // metadata block of one slot: slots int64 [S] | lengths int32 [S] |
   // updates int32 [S][3] | pairs int32 [S][2]
@@ -141,7 +140,6 @@ pa_status pa_engine_create(pa_pool* pool, int32_t* host_tables, int32_t* host_le
   e->kv_row = static_cast<size_t>(num_kv_heads) * head_dim * es;
   e->meta_bytes = 32 * static_cast<size_t>(num_seqs);
   e->ws_bytes = ws_bytes;
-  e->old_entry.resize(num_seqs);
 
   const size_t q_bytes = round256(e->q_row * num_seqs);
   const size_t kv_bytes = round256(e->kv_row * num_seqs);
@@ -218,31 +216,17 @@ pa_status pa_engine_step(pa_engine* e, int32_t row0, int32_t num_rows, const voi
   const int32_t MB = e->MB;
   int32_t* tables = e->h_tables + static_cast<int64_t>(row0) * MB;
   int32_t* lens = e->h_lens + row0;
-  for (int32_t i = 0; i < num_rows; ++i) {
-    const int32_t col = lens[i] / bs;
-    e->old_entry[i] = (lens[i] >= 0 && col < MB) ? tables[static_cast<int64_t>(i) * MB + col] : -1;
-  }
   unsigned char* hm = e->hmeta[b];
   int64_t* slots = reinterpret_cast<int64_t*>(hm);
   int32_t* h_lens_meta = reinterpret_cast<int32_t*>(hm + e->off_lens());
   int32_t* upd = reinterpret_cast<int32_t*>(hm + e->off_upd());
   int32_t* pairs = reinterpret_cast<int32_t*>(hm + e->off_pairs());
-  int32_t npairs = 0;
-  // all or nothing: on failure the pool, tables and lengths are unchanged
-  pa_status st = pa_reserve_slots(e->pool, tables, MB, lens, num_rows, slots, pairs, &npairs);
+  int32_t npairs = 0, nupd = 0;
+  // all or nothing: on failure the pool, tables and lengths are unchanged;
+  // the table entries the reservation wrote go to the device tables below
+  pa_status st = pa_reserve_slots_with_updates(e->pool, tables, MB, lens, num_rows, row0, slots, pairs, &npairs,
+                                               upd, &nupd);
   if (st != PA_OK) return st;
-  int32_t nupd = 0;
-  for (int32_t i = 0; i < num_rows; ++i) {
-    const int32_t pos = lens[i] - 1;   // the reserved token
-    const int32_t col = pos / bs;
-    const int32_t now = tables[static_cast<int64_t>(i) * MB + col];
-    if (pos % bs == 0 || now != e->old_entry[i]) {
-      upd[3 * nupd] = row0 + i;
-      upd[3 * nupd + 1] = col;
-      upd[3 * nupd + 2] = now;
-      ++nupd;
-    }
-  }
   std::memcpy(h_lens_meta, e->h_lens, sizeof(int32_t) * e->S);
 
   unsigned char* dm = e->dmeta[b];

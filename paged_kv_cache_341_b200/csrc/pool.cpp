@@ -205,13 +205,14 @@ pa_status pa_seq_reserve_slot(pa_pool* pool, int32_t* table, int32_t table_cap, 
   return st == PA_OK ? pa::ok() : st;
 }
 
-pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, int32_t* lens, int32_t num_seqs,
-                           int64_t* slots_out, int32_t* pairs_out, int32_t* num_pairs_out) {
-  if (!pool || num_seqs < 0 || table_cap < 0 || !num_pairs_out ||
-      (num_seqs > 0 && (!tables || !lens || !slots_out || !pairs_out)))
+pa_status pa_reserve_slots_with_updates(pa_pool* pool, int32_t* tables, int32_t table_cap, int32_t* lens,
+                                        int32_t num_seqs, int32_t row0, int64_t* slots_out, int32_t* pairs_out,
+                                        int32_t* num_pairs_out, int32_t* updates_out, int32_t* num_updates_out) {
+  if (!pool || num_seqs < 0 || table_cap < 0 || !num_pairs_out || row0 < 0 ||
+      (num_seqs > 0 && (!tables || !lens || !slots_out || !pairs_out)) || (updates_out && !num_updates_out))
     return pa::fail(PA_ERR_INVALID, "pa_reserve_slots: bad argument");
   std::vector<Undo> undo(num_seqs);
-  int32_t npairs = 0;
+  int32_t npairs = 0, nupd = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
     int32_t src, dst;
     int32_t* table = tables + static_cast<int64_t>(s) * table_cap;
@@ -226,9 +227,24 @@ pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, in
       pairs_out[2 * npairs + 1] = dst;
       ++npairs;
     }
+    // the reservation wrote a table entry exactly when it took a block: a
+    // fresh one at offset 0, or the copy of a shared one
+    if (updates_out && undo[s].taken >= 0) {
+      updates_out[3 * nupd] = row0 + s;
+      updates_out[3 * nupd + 1] = undo[s].logical;
+      updates_out[3 * nupd + 2] = table[undo[s].logical];
+      ++nupd;
+    }
   }
   *num_pairs_out = npairs;
+  if (num_updates_out) *num_updates_out = nupd;
   return pa::ok();
+}
+
+pa_status pa_reserve_slots(pa_pool* pool, int32_t* tables, int32_t table_cap, int32_t* lens, int32_t num_seqs,
+                           int64_t* slots_out, int32_t* pairs_out, int32_t* num_pairs_out) {
+  return pa_reserve_slots_with_updates(pool, tables, table_cap, lens, num_seqs, 0, slots_out, pairs_out,
+                                       num_pairs_out, nullptr, nullptr);
 }
 
 }  // extern "C"

@@ -40,6 +40,7 @@ SIGNATURES = {
     "pa_pool_export": (_i32, [_vp, _p32, _p32, _p32]),
     "pa_seq_reserve_slot": (_i32, [_vp, _p32, _i32, _p32, _p64, _p32, _p32]),
     "pa_reserve_slots": (_i32, [_vp, _p32, _i32, _p32, _i32, _p64, _p32, _p32]),
+    "pa_reserve_slots_with_updates": (_i32, [_vp, _p32, _i32, _p32, _i32, _i32, _p64, _p32, _p32, _p32, _p32]),
     "pa_pool_enable_prefix_cache": (_i32, [_vp]),
     "pa_seq_alloc_prompt": (_i32, [_vp, _p32, _i32, _p32, _i32, _p32]),
     "pa_pool_cached_blocks": (_i32, [_vp, _p32]),
@@ -204,6 +205,26 @@ class Pool:
                                      lens.ctypes.data_as(_p32), s, slots.ctypes.data_as(_p64),
                                      pairs.ctypes.data_as(_p32), ctypes.byref(npairs)))
         return slots, pairs[: npairs.value].copy()
+
+    def pa_reserve_slots_with_updates(self, tables, lens, row0, slots_out, pairs_out, updates_out):
+        """``pa_reserve_slots`` writing into caller arrays, also listing the table entries it wrote.
+
+        ``slots_out`` int64 [S], ``pairs_out`` int32 [>=S, 2], ``updates_out`` int32 [>=S, 3] (each
+        contiguous, e.g. views of pinned staging); returns (number of pairs, number of updates).
+        """
+        if tables.dtype != np.int32 or lens.dtype != np.int32 or not tables.flags.c_contiguous:
+            raise TypeError("tables and lens must be contiguous int32 arrays")
+        s = lens.size
+        for a, dt, w in ((slots_out, np.int64, 1), (pairs_out, np.int32, 2), (updates_out, np.int32, 3)):
+            if a.dtype != dt or not a.flags.c_contiguous or a.size < w * s:
+                raise TypeError("output arrays: contiguous, of the right type and size")
+        npairs, nupd = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.pa_reserve_slots_with_updates(self._h, tables.ctypes.data_as(_p32), tables.shape[1],
+                                                  lens.ctypes.data_as(_p32), s, int(row0),
+                                                  slots_out.ctypes.data_as(_p64), pairs_out.ctypes.data_as(_p32),
+                                                  ctypes.byref(npairs), updates_out.ctypes.data_as(_p32),
+                                                  ctypes.byref(nupd)))
+        return npairs.value, nupd.value
 
 
     # -- prefix caching ------------------------------------------------------

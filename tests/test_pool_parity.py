@@ -169,3 +169,53 @@ def test_workload_tables_match_at_full_size(pa):
         need = -(-int(n) // w.block_size)
         assert list(lp.pa_pool_alloc(need)) == op.alloc(need)
     assert state_equal(lp, op)
+
+
+def test_reservation_lists_exactly_the_entries_it_wrote(pa):
+    """pa_reserve_slots_with_updates: slots and pairs as the oracle's reservations, and the
+    (row, column, id) list equal to a diff of the host tables before and after the step."""
+    rng = np.random.default_rng(17)
+    for trial in range(20):
+        bs = int(rng.choice([1, 4, 16]))
+        s = int(rng.integers(1, 12))
+        cap = 24
+        nb = s * cap + 8
+        order = rng.permutation(nb)
+        lp, op = pa.Pool(nb, bs, order), OraclePool(nb, bs, order)
+        tables = np.full((s, cap), -1, np.int32)
+        lens = np.zeros(s, np.int32)
+        otables, olens = [[] for _ in range(s)], [0] * s
+        for r in range(s):
+            target = int(rng.integers(0, cap * bs // 2))
+            for _ in range(target):
+                _, lens[r], _, _ = lp.pa_seq_reserve_slot(tables[r], lens[r])
+                _, olens[r], _, _ = op.reserve_slot(otables[r], olens[r])
+        # some rows become forks of their neighbour (shared blocks -> copy-on-write)
+        for r in range(1, s):
+            if rng.random() < 0.4 and lens[r - 1] > 0:
+                n = -(-int(lens[r - 1]) // bs)
+                lp.pa_pool_free(tables[r, :-(-int(lens[r]) // bs)]) if lens[r] else None
+                op.free(otables[r]) if otables[r] else None
+                lp.pa_pool_fork(tables[r - 1, :n])
+                op.fork(otables[r - 1])
+                tables[r] = tables[r - 1]
+                lens[r] = lens[r - 1]
+                otables[r], olens[r] = list(otables[r - 1]), olens[r - 1]
+        row0 = int(rng.integers(0, 5))
+        for step in range(int(rng.integers(1, 2 * bs + 2))):
+            before = tables.copy()
+            slots = np.empty(s, np.int64)
+            pairs = np.empty((s, 2), np.int32)
+            upd = np.full((s, 3), -7, np.int32)
+            npairs, nupd = lp.pa_reserve_slots_with_updates(tables, lens, row0, slots, pairs, upd)
+            opairs = []
+            for r in range(s):
+                oslot, olens[r], src, dst = op.reserve_slot(otables[r], olens[r])
+                assert slots[r] == oslot
+                if src >= 0:
+                    opairs.append((src, dst))
+            assert [tuple(p) for p in pairs[:npairs]] == opairs
+            rows, cols = np.nonzero(tables != before)
+            expect = sorted((int(r) + row0, int(c), int(tables[r, c])) for r, c in zip(rows, cols))
+            assert sorted(tuple(int(x) for x in u) for u in upd[:nupd]) == expect
+            assert list(lens) == olens and state_equal(lp, op)
