@@ -73,7 +73,7 @@ struct DecodeParams {
   void* out;                     // [S][Hq][D]
   float* part_acc;               // [S][Hq][NP][D]   (partitioned mode)
   float2* part_ml;               // [S][Hq][NP]      (m in base-2 units, l)
-  int* sched;                    // [0]: unit counter, [1]: number of planned units (plan_kernel)
+  int* sched;                    // [0] unit counter, [1] planned units, [2] CTAs that take units (plan_kernel)
   const int4* units;             // planned unit list {seq, part, tile, len}, or null: walk the sequences
   int table_stride;              // elements between rows of block_tables (>= max_blocks)
   int part_offset;               // partial index of partition 0 (shared-prefix mode)
@@ -243,9 +243,10 @@ __device__ __forceinline__ void run_producer(Pipeline<T, D, G>& pl, const Decode
   };
   if (planned) {
     wait_prerequisite_grids();                       // the plan is complete and visible
-    if (lane == 0) total_units = __ldcg(prm.sched + 1);
+    // CTAs beyond the planner's working grid take no units
+    if (lane == 0) total_units = static_cast<int>(blockIdx.x) < __ldcg(prm.sched + 2) ? __ldcg(prm.sched + 1) : 0;
     total_units = __shfl_sync(0xffffffffu, total_units, 0);
-    next_desc = claim();
+    if (total_units > 0) next_desc = claim();
   }
   int rr = blockIdx.x;
 
@@ -937,8 +938,11 @@ __global__ void __maxnreg__(128)
 struct PlanParams {
   const int32_t* context_lens;
   int4* units;                   // entries {seq, part, 0, len}, one per (sequence, partition)
-  int* header;                   // [0] unit counter (zeroed), [1] unit count (entries x num_tiles)
+  int* header;                   // [0] unit counter (zeroed), [1] unit count (entries x num_tiles),
+                                 // [2] decode CTAs that take units
   int num_seqs, partition_size, num_tiles, cap;
+  int num_ctas;                  // CTAs of the decode grid
+  int balance;                   // size the working grid to whole waves of the largest unit
 };
 
 constexpr int kPlanThreads = 1024;
@@ -996,8 +1000,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
     const int chunks = (rem + kChunkTokens - 1) / kChunkTokens;
     return chunks < kPlanBuckets ? chunks : kPlanBuckets - 1;
   };
-  // pass 0: full partitions, and the remainder histogram
+  __shared__ int s_work, s_umax;
+  if (tid == 0) {
+    s_work = 0;
+    s_umax = 1;
+  }
+  // pass 0: full partitions, and the remainder histogram; work in 16-token
+  // chunks per KV-head tile (total and largest unit)
   int written = 0;
+  int my_work = 0, my_umax = 0;
   for (int base = 0; base < S; base += kPlanThreads) {
     const int s = base + tid;
     int len = 0, nfull = 0;
@@ -1006,6 +1017,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
       nfull = P > 0 ? len / P : 0;
       const int b = rem_bucket(len);
       if (b >= 0) atomicAdd(&bucket[b], 1);
+      const int full_chunks = P / kChunkTokens;
+      const int rem_chunks = b >= 0 ? max(1, ((P > 0 ? len % P : len) + kChunkTokens - 1) / kChunkTokens) : 0;
+      my_work += nfull * full_chunks + rem_chunks;
+      my_umax = max(my_umax, max(nfull > 0 ? full_chunks : 0, rem_chunks));
     }
     int round_total;
     const int off = block_exclusive_scan(nfull, warp_sums, &round_total);
@@ -1032,10 +1047,29 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
       bucket[b] = written + run;                  // becomes the cursor of bucket b
       run += c;
     }
+    atomicAdd(&s_work, my_work);
+    atomicMax(&s_umax, my_umax);
     __syncthreads();
     if (tid == 0) {
       prm.header[0] = 0;
       prm.header[1] = (written + tot) * nt;
+      // With units of equal size u, dynamic claiming by A CTAs ends after
+      // ceil(U / A) rounds, while HBM is shared by whichever CTAs are still
+      // busy: a last round that only some CTAs reach runs at the same
+      // per-CTA rate and wastes the rest.  So take k = ceil(U_eff / CTAs)
+      // rounds and A = ceil(U_eff / k) CTAs, U_eff = work / largest unit,
+      // keeping at least 7/8 of the grid busy (HBM stays saturated).
+      int active = prm.num_ctas;
+      if (prm.balance) {
+        const long long work = static_cast<long long>(s_work) * nt;
+        const long long ueff = (work + s_umax - 1) / s_umax;
+        const long long k = (ueff + prm.num_ctas - 1) / prm.num_ctas;
+        long long a = k > 0 ? (ueff + k - 1) / k : prm.num_ctas;
+        const int floor_ctas = prm.num_ctas - prm.num_ctas / 8;
+        a = a < floor_ctas ? floor_ctas : (a > prm.num_ctas ? prm.num_ctas : a);
+        active = static_cast<int>(a);
+      }
+      prm.header[2] = active;
     }
   }
   // pass 1: remainder partitions into their buckets
@@ -1051,11 +1085,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
 
 // ===========================================================================
 // Merge of per-partition partials: M = max m_p, w_p = 2^(m_p - M),
-// out = sum_p w_p acc_p / sum_p w_p l_p.  One warp per (sequence, query
-// head); sequences that fit one partition were written by the decode kernel
-// and are skipped.  Launched as a programmatic dependent of the decode kernel:
-// it waits (griddepcontrol.wait) until that grid has finished and its writes
-// are visible before reading anything it wrote.
+// out = sum_p w_p acc_p / sum_p w_p l_p.  A CTA of 8 warps covers 8 / W query
+// heads of one sequence with W warps per head (W from the partition count the
+// workspace allows: 1 up to 8 partitions, up to 8 for 33 or more); the W warps
+// of a head each take every W-th partition with four rows in flight, and sum
+// their parts through shared memory.  Sequences that fit one partition were
+// written by the decode kernel and are skipped.  Launched as a programmatic
+// dependent of the decode kernel: it reads nothing before griddepcontrol.wait
+// has returned, i.e. before that grid (and so everything before it on the
+// stream) has finished and its writes are visible.
 // ===========================================================================
 struct ReduceParams {
   const int32_t* context_lens;
@@ -1064,67 +1102,88 @@ struct ReduceParams {
   void* out;
   int num_seqs, num_q_heads, partition_size, max_parts, cap;
   int part_offset;               // partials before partition 0 (shared-prefix splits); 0 otherwise
+  int warps_per_head;            // 1, 2, 4 or 8
 };
 
 constexpr int kReduceWarps = 8;
+
+// Warps per (sequence, head) for a partition count: about eight partitions per warp.
+__host__ __device__ constexpr int reduce_warps_per_head(int max_parts) {
+  return max_parts <= 8 ? 1 : (max_parts <= 16 ? 2 : (max_parts <= 32 ? 4 : 8));
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceParams prm) {
   constexpr int PER = D / 32;                // contiguous elements per lane
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
+  __shared__ float2 s_sum[kReduceWarps][D / 2];
   const int s = blockIdx.y;
   wait_prerequisite_grids();                 // the decode grid (and all before it) is done and visible
   int len = prm.context_lens[s];
   len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
   const int np = prm.part_offset + parts_of(len, prm.partition_size);
-  if (prm.part_offset == 0 && np <= 1) return;
+  if (prm.part_offset == 0 && np <= 1) return;          // the same for the whole CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hq = blockIdx.x * kReduceWarps + warp;
-  if (hq >= prm.num_q_heads) return;
-  const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + hq) * prm.max_parts;
-  // lane p holds partition p's (m, l) (partitions beyond 32 fold into lanes)
-  float mx = -INFINITY;
-  for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (mx == -INFINITY) mx = 0.f;            // no partition saw a token: all weights are 0
-  float lsum = 0.f;
-  for (int p = lane; p < np; p += 32) {
-    const float2 ml = prm.part_ml[base + p];
-    lsum += ml.y * exp2_approx(ml.x - mx);
-  }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  const int wph = prm.warps_per_head;
+  const int hq = blockIdx.x * (kReduceWarps / wph) + warp / wph;
+  const int sub = warp & (wph - 1);
+  const bool active = hq < prm.num_q_heads;
+  const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + (active ? hq : 0)) * prm.max_parts;
   float2 o[PER / 2];
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
-  for (int p0 = 0; p0 < np; p0 += 32) {
-    const int pl = p0 + lane;
-    const float wl = pl < np ? exp2_approx(prm.part_ml[base + pl].x - mx) : 0.f;
-    const int n = min(32, np - p0);
-    int k = 0;
-    for (; k + 4 <= n; k += 4) {            // four partitions' loads in flight at once
+  float mx = -INFINITY, lsum = 0.f;
+  if (active) {
+    // every warp of the head computes M and L over all partitions (np (m, l) pairs)
+    for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
+    for (int p = lane; p < np; p += 32) {
+      const float2 ml = prm.part_ml[base + p];
+      lsum += ml.y * exp2_approx(ml.x - mx);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    // this warp's partitions sub, sub + wph, ...: four rows in flight
+    auto row = [&](int p) { return reinterpret_cast<const float2*>(prm.part_acc + (base + p) * D + lane * PER); };
+    int p = sub;
+    for (; p + 3 * wph < np; p += 4 * wph) {
       float2 v[4][PER / 2];
+      float w[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + k + u) * D + lane * PER);
+        const float2* src = row(p + u * wph);
 #pragma unroll
         for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+        w[u] = prm.part_ml[base + p + u * wph].x;
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float w = __shfl_sync(0xffffffffu, wl, k + u);
+        const float wu = exp2_approx(w[u] - mx);
 #pragma unroll
-        for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(w, w), v[u][e]);
+        for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
       }
     }
-    for (; k < n; ++k) {
-      const float w = __shfl_sync(0xffffffffu, wl, k);
-      const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + k) * D + lane * PER);
+    for (; p < np; p += wph) {
+      const float2* src = row(p);
+      const float wu = exp2_approx(prm.part_ml[base + p].x - mx);
 #pragma unroll
-      for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(w, w), src[e]);
+      for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), src[e]);
     }
   }
+  if (wph > 1) {
+#pragma unroll
+    for (int e = 0; e < PER / 2; ++e) s_sum[warp][lane * (PER / 2) + e] = o[e];
+    __syncthreads();
+    if (sub == 0) {
+      for (int k = 1; k < wph; ++k) {
+#pragma unroll
+        for (int e = 0; e < PER / 2; ++e) fadd2(o[e], s_sum[warp + k][lane * (PER / 2) + e]);
+      }
+    }
+  }
+  if (!active || sub != 0) return;
   const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
   T* dst = static_cast<T*>(prm.out) + (static_cast<size_t>(s) * prm.num_q_heads + hq) * D + lane * PER;
 #pragma unroll

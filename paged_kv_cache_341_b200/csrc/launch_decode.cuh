@@ -267,6 +267,8 @@ pa_status launch_decode(const DecodeArgs& a) {
     pp.partition_size = a.P;
     pp.num_tiles = n_tiles;
     pp.cap = a.max_blocks * a.BS;
+    pp.num_ctas = grid;
+    pp.balance = env_int("PA_DECODE_NO_BALANCE") ? 0 : 1;
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -307,9 +309,11 @@ pa_status launch_decode(const DecodeArgs& a) {
     rp.max_parts = np;
     rp.cap = a.max_blocks * a.BS;
     rp.part_offset = a.part_offset;
+    rp.warps_per_head = pa::reduce_warps_per_head(np);
+    const int heads_per_cta = pa::kReduceWarps / rp.warps_per_head;
     // programmatic dependent launch: resident early, waits for the decode grid
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((a.Hq + pa::kReduceWarps - 1) / pa::kReduceWarps, a.S);
+    cfg.gridDim = dim3((a.Hq + heads_per_cta - 1) / heads_per_cta, a.S);
     cfg.blockDim = dim3(pa::kReduceWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = a.stream;

@@ -64,17 +64,6 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// d += a on a pair of float32 lanes (one instruction on sm_100a).
-__device__ __forceinline__ void fadd2(float2& d, const float2 a) {
-  asm("{\n\t.reg .b64 rd, ra;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rd, {%0, %1};\n\t"
-      "add.rn.f32x2 rd, rd, ra;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d.x), "+f"(d.y)
-      : "f"(a.x), "f"(a.y));
-}
-
 // 4-D tile load global -> shared through a tensor map, completing on `bar`.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
                                             int c3) {

@@ -153,6 +153,17 @@ __device__ __forceinline__ void ffma2(float2& d, const float2 a, const float2 b)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
 }
 
+// d += a on a pair of float32 lanes (one instruction on sm_100a).
+__device__ __forceinline__ void fadd2(float2& d, const float2 a) {
+  asm("{\n\t.reg .b64 rd, ra;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(a.x), "f"(a.y));
+}
+
 // d = d * s on a pair of float32 lanes.
 __device__ __forceinline__ void fmul2(float2& d, const float2 s) {
   asm("{\n\t.reg .b64 rd, rs;\n\t"
