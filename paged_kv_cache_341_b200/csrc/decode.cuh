@@ -1058,9 +1058,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
       // busy: a last round that only some CTAs reach runs at the same
       // per-CTA rate and wastes the rest.  So take k = ceil(U_eff / CTAs)
       // rounds and A = ceil(U_eff / k) CTAs, U_eff = work / largest unit,
-      // keeping at least 7/8 of the grid busy (HBM stays saturated).
+      // keeping at least 7/8 of the grid busy (HBM stays saturated).  Only
+      // when the smaller remainder units are too few to fill that last round
+      // (fewer than one per CTA); otherwise they already do.
       int active = prm.num_ctas;
-      if (prm.balance) {
+      if (prm.balance && static_cast<long long>(tot) * nt < prm.num_ctas) {
         const long long work = static_cast<long long>(s_work) * nt;
         const long long ueff = (work + s_umax - 1) / s_umax;
         const long long k = (ueff + prm.num_ctas - 1) / prm.num_ctas;

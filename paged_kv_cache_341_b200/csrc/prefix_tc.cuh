@@ -11,33 +11,35 @@
 // tensor cores are for.  The producer also brings in the query tiles by TMA.
 //
 // Roles (320 threads):
-//   warp 0     TMA producer: 128-token K and V tiles of the prefix, straight
+//   warp 0     TMA producer: 64-token K and V tiles of the prefix, straight
 //              from the paged cache through the block list, into two rings
-//              of `stages` 128-byte-swizzled tiles ([D/64 panels][128 tok][128 B]);
+//              of `stages` 128-byte-swizzled tiles ([D/64 panels][64 tok][128 B]);
 //              each tile serves both query tiles.
 //   warp 1     allocates all 512 tensor-memory columns; lane 0 issues the
-//              MMAs, for query tile g (columns 256g..256g+255):
-//                S_g  = Q_g K_t^T  (M 128, N 128, K = D; columns 0..127)
-//                O_g += P_g V_t    (M 128, N = D, K 128; P read from tensor
-//                                   memory where S was, O in columns 128..)
-//              in the order PV_0(t), S_0(t+1), PV_1(t), S_1(t+1), so that
-//              each softmax group has the other group's products to hide
-//              behind, and tracks completion with tcgen05.commit.
+//              MMAs.  Query tile g owns columns 256g..256g+255: two S buffers
+//              (0..63, 64..127) and O (128..255).  Token tile t of query tile g:
+//                S_g(t)  = Q_g K_t^T  (M 128, N 64, K = D) into buffer t % 2
+//                O_g    += P_g(t) V_t (M 128, N = D, K 64; P read from tensor
+//                                      memory where S_g(t) was)
+//              S is double-buffered, so S_g(t+1) is computed while the softmax
+//              works on S_g(t): the MMAs are issued as PV_g(t), S_g(t+2) once
+//              P_g(t) is ready, and the softmax never waits for the tensor
+//              core unless the tensor core is the bottleneck.
 //   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1; one query
-//              row per thread (tensor-memory lane): one pass over S in
-//              32-column chunks (the next chunk's load in flight), online max
-//              with the decode kernel's threshold rule chunk by chunk (the
-//              reference moves only when a score passes it by 2^8; O and the
-//              tile's stored P chunks are then rescaled in tensor memory),
-//              P = 2^(s*scale*log2(e) - m) rounded to the cache's 16-bit type
-//              and stored back into tensor memory over S as the A operand of
-//              the next product; l sums the rounded weights.
+//              row per thread (tensor-memory lane).  Per token tile: the 64
+//              scores in registers (loaded while the previous tile's weights
+//              were computed), their maximum, the decode kernel's threshold
+//              rule for the reference maximum (it moves only when a scaled
+//              score passes it by 2^8; O is then rescaled in tensor memory
+//              after PV_g(t-1) has completed), P = 2^(s*scale*log2(e) - m)
+//              rounded to the cache's 16-bit type and stored over S as the A
+//              operand of PV; l sums the rounded weights.
 // Products issued by one thread run in issue order, and a commit arrives only
-// once everything issued before it has completed.  So S(t+1) may overwrite
-// P(t) as soon as PV(t) is issued, and when S(t) is reported ready, PV(t-1)
-// has completed and O may be rescaled.  Q is loaded once per CTA (rows beyond
-// the batch are zero; a second tile with no rows at all is skipped).  Every wait is bounded in time; on a timeout all roles
-// fall through to the end, the MMA issuer waits for its own products, and the
+// once everything issued before it has completed: S_g(t+2) overwrites P_g(t)
+// only after PV_g(t), which was issued before it, has read it.  Q is loaded
+// once per CTA (rows beyond the batch are zero; a second tile with no rows at
+// all is skipped).  Every wait is bounded in time; on a timeout all roles fall
+// through to the end, the MMA issuer waits for its own products, and the
 // tensor memory is released before the CTA exits.
 #ifndef PAGEDATTN_PREFIX_TC_CUH
 #define PAGEDATTN_PREFIX_TC_CUH
@@ -76,15 +78,25 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
 
 constexpr int kUmmaRows = 128;        // query rows per tile (MMA M)
 constexpr int kUmmaTiles = 2;         // query tiles per CTA
-constexpr int kUmmaTile = 128;        // prefix tokens per stage (MMA N of S, K of PV)
+constexpr int kUmmaTile = 64;         // prefix tokens per stage (MMA N of S, K of PV)
 constexpr int kUmmaThreads = 64 + kUmmaTiles * 128;   // producer, MMA, softmax groups
 constexpr uint32_t kUmmaTmemCols = 512;
+constexpr uint32_t kUmmaGroupCols = 256;              // per query tile: S buffers 0..127, O 128..255
+constexpr int kGroupBars = 7;                         // mbarriers per query tile
+// At least half of an SM's shared memory, so that one CTA holds the SM (and
+// all of its tensor memory) whatever the head size.
+constexpr size_t kUmmaMinSmem = 120 * 1024;
+
+template <int D>
+__host__ __device__ constexpr size_t prefix_umma_layout_bytes(int stages) {
+  return kSmemAlign + kUmmaTiles * static_cast<size_t>(D / 64) * kUmmaRows * 128          // Q panels
+         + 2 * static_cast<size_t>(stages) * (D / 64) * kUmmaTile * 128                  // K and V rings
+         + (4 * static_cast<size_t>(stages) + kGroupBars * kUmmaTiles + 1) * sizeof(uint64_t) + 16;
+}
 
 template <int D>
 __host__ __device__ constexpr size_t prefix_umma_smem_bytes(int stages) {
-  return kSmemAlign + kUmmaTiles * static_cast<size_t>(D / 64) * kUmmaRows * 128   // Q panels
-         + 2 * static_cast<size_t>(stages) * (D / 64) * kUmmaTile * 128              // K and V rings
-         + (4 * static_cast<size_t>(stages) + 4 * kUmmaTiles + 1) * sizeof(uint64_t) + 16;
+  return prefix_umma_layout_bytes<D>(stages) < kUmmaMinSmem ? kUmmaMinSmem : prefix_umma_layout_bytes<D>(stages);
 }
 
 template <typename T, int D, int G>
@@ -94,10 +106,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   static_assert(sizeof(T) == 2, "tensor-core path takes 16-bit caches");
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kHalves = D / 64;                        // 128-byte panels per row
-  constexpr uint32_t kPanel = kUmmaTile * 128;           // one panel of a K/V tile (16 KB)
+  constexpr uint32_t kPanel = kUmmaTile * 128;           // one panel of a K/V tile (8 KB)
   constexpr uint32_t kTileBytes = kHalves * kPanel;      // K (or V) bytes per stage
   constexpr uint32_t kQPanel = kUmmaRows * 128;          // one panel of Q (16 KB)
   constexpr uint32_t kQBytes = kHalves * kQPanel;        // one query tile
+  constexpr int kS = kUmmaTile;                          // scores per row and tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   using M = MmaType<T>;
 
@@ -113,13 +126,17 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   uint64_t* k_empty = k_full + stages;
   uint64_t* v_full = k_empty + stages;
   uint64_t* v_empty = v_full + stages;
-  // per query tile g, 4 barriers at grp + 4g: s_full, p_full, o_done, q_full
+  // per query tile g, kGroupBars barriers at grp + kGroupBars * g: s_full and
+  // p_full of S buffers 0 and 1 (the softmax may finish tile t + 1 before
+  // the MMA issuer has taken tile t, so P readiness alternates buffers too),
+  // pv_done (every PV), o_done (the last PV), q_full
   uint64_t* grp = v_empty + stages;
-  auto s_full = [&](int g) { return grp + 4 * g; };
-  auto p_full = [&](int g) { return grp + 4 * g + 1; };
-  auto o_done = [&](int g) { return grp + 4 * g + 2; };
-  auto q_full = [&](int g) { return grp + 4 * g + 3; };
-  uint64_t* drain = grp + 4 * kUmmaTiles;
+  auto s_full = [&](int g, int b) { return grp + kGroupBars * g + b; };
+  auto p_full = [&](int g, int b) { return grp + kGroupBars * g + 2 + b; };
+  auto pv_done = [&](int g) { return grp + kGroupBars * g + 4; };
+  auto o_done = [&](int g) { return grp + kGroupBars * g + 5; };
+  auto q_full = [&](int g) { return grp + kGroupBars * g + 6; };
+  uint64_t* drain = grp + kGroupBars * kUmmaTiles;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -144,8 +161,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     // softmax-side barriers take one arrival per warp (elected lane after __syncwarp)
     for (int g = 0; g < kUmmaTiles; ++g) {
-      mbar_init(s_full(g), 1);
-      mbar_init(p_full(g), 4);
+      mbar_init(s_full(g, 0), 1);
+      mbar_init(s_full(g, 1), 1);
+      mbar_init(p_full(g, 0), 4);
+      mbar_init(p_full(g, 1), 4);
+      mbar_init(pv_done(g), 1);
       mbar_init(o_done(g), 1);
       mbar_init(q_full(g), 1);
     }
@@ -187,9 +207,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     for (int t = 0; t < ntiles; ++t) {
       const int tok0 = tok_lo + t * kUmmaTile;
       const int ntok = min(kUmmaTile, tok_hi - tok0);
-      const int npieces = ntok / piece_rows;     // <= 16
+      const int npieces = ntok / piece_rows;     // <= 8
       // one box per lane: piece pc = lane / kHalves, panel hf = lane % kHalves
-      const int nbox = npieces * kHalves;        // <= 32
+      const int nbox = npieces * kHalves;        // <= 16
       const int pc = lane / kHalves;
       const int hf = lane - pc * kHalves;
       int row = 0;
@@ -278,51 +298,63 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       tc::fence_after_sync();
       int kst = 0, vst = 0;
       uint32_t kph = 0, vph = 0;
-      // S_g = Q_g K^T into columns 256g..256g+127
-      auto issue_s = [&](int g, int ks) {
+      // S_g = Q_g K^T into S buffer b of query tile g
+      auto issue_s = [&](int g, int ks, int b) {
         const uint64_t kb = k_desc + ((ks * kTileBytes) >> 4);
         const uint64_t qb = q_desc + ((g * kQBytes) >> 4);
+        const uint32_t d_tmem = tmem + g * kUmmaGroupCols + b * kS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          tc::mma_f16_ss(tmem + g * 256, qb + (((kk >> 2) * kQPanel + (kk & 3) * 32) >> 4),
+          tc::mma_f16_ss(d_tmem, qb + (((kk >> 2) * kQPanel + (kk & 3) * 32) >> 4),
                          kb + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
-        tc::commit(s_full(g));
+        tc::commit(s_full(g, b));
       };
-      // O_g += P_g V; P in columns 256g..256g+63, two 16-bit values per column
-      auto issue_pv = [&](int g, int vs, bool first) {
+      // O_g += P_g V; P in the first 32 columns of S buffer b, two 16-bit values per column
+      auto issue_pv = [&](int g, int vs, int b, bool first) {
         const uint64_t vb = v_desc + ((vs * kTileBytes) >> 4);
+        const uint32_t p_tmem = tmem + g * kUmmaGroupCols + b * kS;
 #pragma unroll
         for (int kk = 0; kk < kUmmaTile / 16; ++kk)
-          tc::mma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8, vb + ((kk * 16 * 128) >> 4), idesc_o,
+          tc::mma_f16_ts(tmem + g * kUmmaGroupCols + 128, p_tmem + kk * 8, vb + ((kk * 16 * 128) >> 4), idesc_o,
                          !first || kk > 0);
+        tc::commit(pv_done(g));
       };
-      if (ok && ntiles > 0) {
+      // S of the first two token tiles
+      for (int t = 0; ok && t < min(2, ntiles); ++t) {
         ok = mbar_wait(&k_full[kst], kph, abort_flag);
-        if (ok) {
-          tc::fence_after_sync();
-          for (int g = 0; g < ngroups; ++g) issue_s(g, kst);
-          tc::commit(&k_empty[kst]);
-          if (++kst == stages) {
-            kst = 0;
-            kph ^= 1;
-          }
+        if (!ok) break;
+        tc::fence_after_sync();
+        for (int g = 0; g < ngroups; ++g) issue_s(g, kst, t);
+        tc::commit(&k_empty[kst]);
+        if (++kst == stages) {
+          kst = 0;
+          kph ^= 1;
         }
       }
       for (int t = 0; ok && t < ntiles; ++t) {
-        const bool more = t + 1 < ntiles;
-        if (!mbar_wait(&v_full[vst], vph, abort_flag) || (more && !mbar_wait(&k_full[kst], kph, abort_flag))) {
+        const bool more = t + 2 < ntiles;
+        if (!mbar_wait(&v_full[vst], vph, abort_flag)) {
           ok = false;
           break;
         }
         for (int g = 0; g < ngroups; ++g) {
           // P_g(t) written (and O rescaled if the maximum moved)
-          if (!mbar_wait(p_full(g), t & 1, abort_flag)) {
+          if (!mbar_wait(p_full(g, t & 1), (t >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          issue_pv(g, vst, t == 0);
-          if (more) issue_s(g, kst);                  // overwrites P_g(t) after PV_g(t) in issue order
+          issue_pv(g, vst, t & 1, t == 0);
+          if (more) {
+            if (g == 0) {
+              if (!mbar_wait(&k_full[kst], kph, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc::fence_after_sync();
+            }
+            issue_s(g, kst, t & 1);                  // buffer of S(t+2) = buffer of P(t), after PV(t)
+          }
         }
         if (!ok) break;
         tc::commit(&v_empty[vst]);
@@ -349,7 +381,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int g = (warp - 2) / 4;                              // query tile of this group
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                       // tensor-memory lane = query row in the tile
-    const uint32_t t_lane = tmem + g * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t t_lane = tmem + g * kUmmaGroupCols + (static_cast<uint32_t>(quarter * 32) << 16);
     const int gr = row0 + g * kUmmaRows + row;
     const bool valid = gr < rows_total;
     const int s_idx = valid ? gr / G : 0;
@@ -359,129 +391,119 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const float2 qk2 = make_float2(qk, qk);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
+
+    // One token tile: `cur` holds its 64 scores; the next tile's scores are
+    // loaded into `nxt` while this tile's weights are computed.
+    auto tile = [&](int t, uint32_t (&cur)[kS], uint32_t (&nxt)[kS]) -> bool {
       const int ntok = min(kUmmaTile, tok_hi - (tok_lo + t * kUmmaTile));
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), t & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      // One pass over S in 32-column chunks, the load of chunk i + 1 in
-      // flight while chunk i is turned into P.  The reference maximum m
-      // follows the threshold rule chunk by chunk: it moves only when a
-      // chunk's scaled maximum passes it by more than 2^8 (the scaled
-      // maximum is max(s) * qk for qk >= 0 and min(s) * qk otherwise;
-      // rounding is monotonic).  When it moves, O (earlier tiles) and the P
-      // chunks of this tile already stored are rescaled.  P = 2^(s*qk - m) is
-      // rounded to T and packed two per column over scores already read;
-      // lt sums this tile's rounded weights.
       const bool full = ntok == kUmmaTile;
-      float lt = 0.f;
-      uint32_t sbuf[2][32];
-      tc::tmem_ld32(t_lane, sbuf[0]);
-      tc::tmem_wait_ld();
+      if (!full) {
 #pragma unroll
-      for (int cb = 0; cb < kUmmaTile / 32; ++cb) {
-        uint32_t (&cur)[32] = sbuf[cb & 1];
-        if (cb + 1 < kUmmaTile / 32) tc::tmem_ld32(t_lane + (cb + 1) * 32, sbuf[(cb + 1) & 1]);
-        // the sign of qk and whether the tile is full are the same for the
-        // whole warp: one tight loop per case
-        if (!full) {
+        for (int j = 0; j < kS; ++j) cur[j] = j < ntok ? cur[j] : __float_as_uint(pad);
+      }
+      // maximum (minimum for a negative scale) of the raw scores: four
+      // chains of three-input max over the 64 scores
+      float cm[4];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) cur[j] = cb * 32 + j < ntok ? cur[j] : __float_as_uint(pad);
-        }
-        // four chains of three-input max (min) over the 32 scores
-        float cm[4];
+      for (int i = 0; i < 4; ++i) cm[i] = __uint_as_float(cur[i]);
+      float ext;
+      if (qk >= 0.f) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cm[i] = __uint_as_float(cur[i]);
-        float ext;
-        if (qk >= 0.f) {
+        for (int j = 4; j < kS - 4; j += 8)
 #pragma unroll
-          for (int j = 4; j < 28; j += 8)
+          for (int k = 0; k < 4; ++k) cm[k] = fmax3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
 #pragma unroll
-            for (int k = 0; k < 4; ++k) cm[k] = fmax3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
+        for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __uint_as_float(cur[kS - 4 + k]));
+        ext = fmax3(fmaxf(cm[0], cm[1]), cm[2], cm[3]);
+      } else {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __uint_as_float(cur[28 + k]));
-          ext = fmax3(fmaxf(cm[0], cm[1]), cm[2], cm[3]);
-        } else {
+        for (int j = 4; j < kS - 4; j += 8)
 #pragma unroll
-          for (int j = 4; j < 28; j += 8)
+          for (int k = 0; k < 4; ++k) cm[k] = fmin3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
 #pragma unroll
-            for (int k = 0; k < 4; ++k) cm[k] = fmin3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
+        for (int k = 0; k < 4; ++k) cm[k] = fminf(cm[k], __uint_as_float(cur[kS - 4 + k]));
+        ext = fmin3(fminf(cm[0], cm[1]), cm[2], cm[3]);
+      }
+      const float c = ext * qk;
+      if (__any_sync(0xffffffffu, c > m + kTau)) {
+        const float mn = c > m + kTau ? c : m;
+        const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
+        if (t >= 1) {
+          // O holds PV(0..t-1): wait until PV(t-1) has completed (PV(t)
+          // waits for this tile's P), then rescale it in tensor memory
+          if (!__all_sync(0xffffffffu, mbar_wait(pv_done(g), (t - 1) & 1, abort_flag))) return false;
+          tc::fence_after_sync();
+#pragma unroll 1
+          for (int ob = 0; ob < D / 16; ++ob) {
+            uint32_t o[16];
+            tc::tmem_ld16(t_lane + 128 + ob * 16, o);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) cm[k] = fminf(cm[k], __uint_as_float(cur[28 + k]));
-          ext = fmin3(fminf(cm[0], cm[1]), cm[2], cm[3]);
-        }
-        const float c = ext * qk;
-        if (__any_sync(0xffffffffu, c > m + kTau)) {
-          const float mn = c > m + kTau ? c : m;
-          const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
-          if (t >= 1) {
-            // earlier tiles' O: PV(t-1) has completed (S(t) was issued after
-            // it) and PV(t) waits for this tile's P
-#pragma unroll
-            for (int ob = 0; ob < D / 32; ++ob) {
-              uint32_t o[32];
-              tc::tmem_ld32(t_lane + 128 + ob * 32, o);
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-              tc::tmem_st32(t_lane + 128 + ob * 32, o);
-            }
+            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+            tc::tmem_st16(t_lane + 128 + ob * 16, o);
           }
-          if (cb > 0) {
-            // this tile's P chunks stored so far, re-rounded; their sum again
-            tc::tmem_wait_st();
-            lt = 0.f;
-            for (int pb = 0; pb < cb; ++pb) {
-              uint32_t pw[16];
-              tc::tmem_ld16(t_lane + pb * 16, pw);
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 u = M::unpack(pw[i]);
-                pw[i] = M::pack(u.x * f, u.y * f);
-                const float2 r = M::unpack(pw[i]);
-                lt += r.x + r.y;
-              }
-              tc::tmem_st16(t_lane + pb * 16, pw);
-            }
-          }
-          l *= f;
-          m = mn;
         }
-        const float2 nm2 = make_float2(-m, -m);
-        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        l *= f;
+        m = mn;
+      }
+      // the next tile's scores, in flight while this tile's weights are
+      // formed: the first half now, the second once the first half of this
+      // tile's scores is spent (so at most 96 scores are held at a time)
+      const bool has_next = t + 1 < ntiles;
+      const int nb = (t + 1) & 1;
+      if (has_next) {
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full(g, nb), ((t + 1) >> 1) & 1, abort_flag))) return false;
+        tc::fence_after_sync();
+        tc::tmem_ld32_at<0>(t_lane + nb * kS, nxt);
+      }
+      // P = 2^(s * qk - m), rounded to T, two per column over this tile's S;
+      // the row sum takes the rounded values
+      const float2 nm2 = make_float2(-m, -m);
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const uint32_t p_col = t_lane + (t & 1) * kS;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (half == 1 && has_next) tc::tmem_ld32_at<32>(t_lane + nb * kS + 32, nxt);
         uint32_t w[16];
-        if (full) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float2 e = nm2;
-            ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
-            w[i] = M::pack(exp2_approx(e.x), exp2_approx(e.y));
-            fadd2(ls[i & 1], M::unpack(w[i]));
+        for (int i = 0; i < 16; ++i) {
+          const int j = half * 32 + 2 * i;
+          float2 e = nm2;
+          ffma2(e, make_float2(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1])), qk2);
+          float p0 = exp2_approx(e.x), p1 = exp2_approx(e.y);
+          if (!full) {
+            p0 = j < ntok ? p0 : 0.f;
+            p1 = j + 1 < ntok ? p1 : 0.f;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = cb * 32 + 2 * i;
-            float2 e = nm2;
-            ffma2(e, make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), qk2);
-            const float p0 = j < ntok ? exp2_approx(e.x) : 0.f;
-            const float p1 = j + 1 < ntok ? exp2_approx(e.y) : 0.f;
-            w[i] = M::pack(p0, p1);
-            fadd2(ls[i & 1], M::unpack(w[i]));
-          }
+          w[i] = M::pack(p0, p1);
+          fadd2(ls[i & 1], M::unpack(w[i]));
         }
-        lt += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
-        tc::tmem_st16(t_lane + cb * 16, w);
-        if (cb + 1 < kUmmaTile / 32) tc::tmem_wait_ld();
+        tc::tmem_st16(p_col + half * 16, w);
       }
       tc::tmem_wait_st();
-      l += lt;
+      l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(g));
+      if (lane == 0) mbar_arrive(p_full(g, t & 1));
+      if (has_next) tc::tmem_wait_ld();
+      return true;
+    };
+
+    uint32_t sa[kS], sb[kS];
+    if (ntiles > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(g, 0), 0, abort_flag));
+      if (ok) {
+        tc::fence_after_sync();
+        tc::tmem_ld32_at<0>(t_lane, sa);
+        tc::tmem_ld32_at<32>(t_lane + 32, sa);
+        tc::tmem_wait_ld();
+      }
+    }
+#pragma unroll 1
+    for (int t = 0; ok && t < ntiles; t += 2) {
+      ok = tile(t, sa, sb);
+      if (!ok || t + 1 >= ntiles) break;
+      ok = tile(t + 1, sb, sa);
     }
     if (ok && ntiles > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done(g), 0, abort_flag))) ok = false;
     tc::fence_after_sync();
