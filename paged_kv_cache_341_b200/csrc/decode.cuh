@@ -929,11 +929,15 @@ __global__ void __maxnreg__(128)
 //
 // It is launched as a programmatic dependent of the kernel before it on the
 // stream and lets the decode grid launch at once (its CTAs set up and then
-// wait for the planner), but it reads and writes nothing before its own
-// griddepcontrol.wait has returned.  That wait matters twice over: the kernel
-// before may be the previous call's decode grid, still claiming units from
-// the same workspace (resetting the counter under it would hand it this
-// call's units), or it may be the kernel that wrote the lengths.
+// wait for the planner), but it writes nothing before its own
+// griddepcontrol.wait has returned, and trusts no length read before it.
+// That wait matters twice over: the kernel before may be the previous call's
+// decode grid, still claiming units from the same workspace (resetting the
+// counter under it would hand it this call's units), or it may be the kernel
+// that wrote the lengths.  For up to 4096 sequences the plan is worked out
+// ahead of the wait from the lengths as they stand, then the lengths are read
+// again after it and the plan is redone if any changed; larger batches wait
+// first.
 // ===========================================================================
 struct PlanParams {
   const int32_t* context_lens;
@@ -976,17 +980,40 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   return before + incl - v;
 }
 
+// Working grid for the decode kernel (written to header[2]): with units of
+// equal size u, dynamic claiming by A CTAs ends after ceil(U / A) rounds,
+// while HBM is shared by whichever CTAs are still busy: a last round that
+// only some CTAs reach runs at the same per-CTA rate and wastes the rest.  So
+// take k = ceil(U_eff / CTAs) rounds and A = ceil(U_eff / k) CTAs, U_eff =
+// work / largest unit, keeping at least 7/8 of the grid busy (HBM stays
+// saturated).  Only when the smaller remainder units are too few to fill
+// that last round (fewer than one per CTA); otherwise they already do.
+__device__ __forceinline__ int plan_working_grid(const PlanParams& prm, int rem_entries, int work_chunks,
+                                                 int largest_chunks) {
+  const int nt = prm.num_tiles;
+  if (!prm.balance || static_cast<long long>(rem_entries) * nt >= prm.num_ctas) return prm.num_ctas;
+  const long long work = static_cast<long long>(work_chunks) * nt;
+  const long long ueff = (work + largest_chunks - 1) / largest_chunks;
+  const long long k = (ueff + prm.num_ctas - 1) / prm.num_ctas;
+  long long a = k > 0 ? (ueff + k - 1) / k : prm.num_ctas;
+  const int floor_ctas = prm.num_ctas - prm.num_ctas / 8;
+  a = a < floor_ctas ? floor_ctas : (a > prm.num_ctas ? prm.num_ctas : a);
+  return static_cast<int>(a);
+}
+
+constexpr int kPlanSpecRounds = 4;     // batches of up to 4 x 1024 sequences are planned ahead of the wait
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm) {
   __shared__ int bucket[kPlanBuckets];
   __shared__ int warp_sums[32];
+  __shared__ int s_work, s_umax;
   allow_dependent_launch();                    // the decode grid may launch; it waits for this one
-  wait_prerequisite_grids();                   // the kernel before has finished and its writes are visible
   const int tid = threadIdx.x;
   const int S = prm.num_seqs, P = prm.partition_size, nt = prm.num_tiles;
-  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) bucket[b] = 0;
-  __syncthreads();
+  const int rounds = (S + kPlanThreads - 1) / kPlanThreads;
+  // lengths through L2 (never a line cached in L1 before the wait)
   auto load_len = [&](int s) {
-    int len = prm.context_lens[s];
+    int len = __ldcg(prm.context_lens + s);
     return len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
   };
   auto rem_bucket = [&](int len) {               // -1: no remainder unit
@@ -1000,35 +1027,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
     const int chunks = (rem + kChunkTokens - 1) / kChunkTokens;
     return chunks < kPlanBuckets ? chunks : kPlanBuckets - 1;
   };
-  __shared__ int s_work, s_umax;
-  if (tid == 0) {
-    s_work = 0;
-    s_umax = 1;
-  }
-  // pass 0: full partitions, and the remainder histogram; work in 16-token
-  // chunks per KV-head tile (total and largest unit)
-  int written = 0;
-  int my_work = 0, my_umax = 0;
-  for (int base = 0; base < S; base += kPlanThreads) {
-    const int s = base + tid;
-    int len = 0, nfull = 0;
-    if (s < S) {
-      len = load_len(s);
-      nfull = P > 0 ? len / P : 0;
-      const int b = rem_bucket(len);
-      if (b >= 0) atomicAdd(&bucket[b], 1);
-      const int full_chunks = P / kChunkTokens;
-      const int rem_chunks = b >= 0 ? max(1, ((P > 0 ? len % P : len) + kChunkTokens - 1) / kChunkTokens) : 0;
-      my_work += nfull * full_chunks + rem_chunks;
-      my_umax = max(my_umax, max(nfull > 0 ? full_chunks : 0, rem_chunks));
-    }
-    int round_total;
-    const int off = block_exclusive_scan(nfull, warp_sums, &round_total);
-    for (int p = 0; p < nfull; ++p) prm.units[written + off + p] = make_int4(s, p, 0, len);
-    written += round_total;
-  }
-  // bucket starts, largest remainders first: start[b] = written + sum_{b' > b} count[b']
-  {
+  const int full_chunks = P / kChunkTokens;
+  auto rem_chunks = [&](int len, int b) {
+    return b >= 0 ? max(1, ((P > 0 ? len % P : len) + kChunkTokens - 1) / kChunkTokens) : 0;
+  };
+  // Bucket starts, largest remainders first: start[b] = written + sum_{b' > b}
+  // count[b'] (each bucket counter becomes the cursor of its bucket).  Returns
+  // the number of remainder entries.
+  auto bucket_starts = [&](int written) {
     constexpr int PER = kPlanBuckets / kPlanThreads;
     int local[PER];
     int sum = 0;
@@ -1042,46 +1048,127 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
     int run = off;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      const int b = kPlanBuckets - 1 - (tid * PER + i);
-      const int c = local[i];
-      bucket[b] = written + run;                  // becomes the cursor of bucket b
-      run += c;
+      bucket[kPlanBuckets - 1 - (tid * PER + i)] = written + run;
+      run += local[i];
     }
+    return tot;
+  };
+  auto reset = [&]() {
+    for (int b = tid; b < kPlanBuckets; b += kPlanThreads) bucket[b] = 0;
+    if (tid == 0) {
+      s_work = 0;
+      s_umax = 1;
+    }
+    __syncthreads();
+  };
+
+  if (rounds > kPlanSpecRounds) {
+    // Large batch: wait for the kernel before first, then plan and write in
+    // one sweep per 1024 sequences.
+    wait_prerequisite_grids();
+    reset();
+    int written = 0, my_work = 0, my_umax = 0;
+    for (int base = 0; base < S; base += kPlanThreads) {
+      const int s = base + tid;
+      int len = 0, nfull = 0;
+      if (s < S) {
+        len = load_len(s);
+        nfull = P > 0 ? len / P : 0;
+        const int b = rem_bucket(len);
+        if (b >= 0) atomicAdd(&bucket[b], 1);
+        my_work += nfull * full_chunks + rem_chunks(len, b);
+        my_umax = max(my_umax, max(nfull > 0 ? full_chunks : 0, rem_chunks(len, b)));
+      }
+      int round_total;
+      const int off = block_exclusive_scan(nfull, warp_sums, &round_total);
+      for (int p = 0; p < nfull; ++p) prm.units[written + off + p] = make_int4(s, p, 0, len);
+      written += round_total;
+    }
+    const int tot = bucket_starts(written);
     atomicAdd(&s_work, my_work);
     atomicMax(&s_umax, my_umax);
     __syncthreads();
     if (tid == 0) {
       prm.header[0] = 0;
       prm.header[1] = (written + tot) * nt;
-      // With units of equal size u, dynamic claiming by A CTAs ends after
-      // ceil(U / A) rounds, while HBM is shared by whichever CTAs are still
-      // busy: a last round that only some CTAs reach runs at the same
-      // per-CTA rate and wastes the rest.  So take k = ceil(U_eff / CTAs)
-      // rounds and A = ceil(U_eff / k) CTAs, U_eff = work / largest unit,
-      // keeping at least 7/8 of the grid busy (HBM stays saturated).  Only
-      // when the smaller remainder units are too few to fill that last round
-      // (fewer than one per CTA); otherwise they already do.
-      int active = prm.num_ctas;
-      if (prm.balance && static_cast<long long>(tot) * nt < prm.num_ctas) {
-        const long long work = static_cast<long long>(s_work) * nt;
-        const long long ueff = (work + s_umax - 1) / s_umax;
-        const long long k = (ueff + prm.num_ctas - 1) / prm.num_ctas;
-        long long a = k > 0 ? (ueff + k - 1) / k : prm.num_ctas;
-        const int floor_ctas = prm.num_ctas - prm.num_ctas / 8;
-        a = a < floor_ctas ? floor_ctas : (a > prm.num_ctas ? prm.num_ctas : a);
-        active = static_cast<int>(a);
-      }
-      prm.header[2] = active;
+      prm.header[2] = plan_working_grid(prm, tot, s_work, s_umax);
     }
+    for (int s = tid; s < S; s += kPlanThreads) {
+      const int len = load_len(s);
+      const int b = rem_bucket(len);
+      if (b < 0) continue;
+      const int pos = atomicAdd(&bucket[b], 1);
+      prm.units[pos] = make_int4(s, P > 0 ? len / P : 0, 0, len);
+    }
+    return;
   }
-  // pass 1: remainder partitions into their buckets
-  for (int s = tid; s < S; s += kPlanThreads) {
-    const int len = load_len(s);
-    const int b = rem_bucket(len);
-    if (b < 0) continue;
-    const int pos = atomicAdd(&bucket[b], 1);
-    const int part = P > 0 ? len / P : 0;
-    prm.units[pos] = make_int4(s, part, 0, len);
+
+  // Up to 4096 sequences: the whole plan is worked out in registers from
+  // lengths read before the kernel before has finished (that kernel may be an
+  // append, which writes no length, or anything else on the stream); after
+  // griddepcontrol.wait the lengths are read again, and if any changed the
+  // plan is worked out once more.  Nothing is written before the wait.
+  int len[kPlanSpecRounds], base_off[kPlanSpecRounds], pos[kPlanSpecRounds];
+  int written = 0, tot = 0;
+  bool waited = false;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    reset();
+    written = 0;
+    int my_work = 0, my_umax = 0;
+#pragma unroll
+    for (int r = 0; r < kPlanSpecRounds; ++r) {
+      if (r >= rounds) break;
+      const int s = r * kPlanThreads + tid;
+      int nfull = 0;
+      len[r] = 0;
+      if (s < S) {
+        len[r] = load_len(s);
+        nfull = P > 0 ? len[r] / P : 0;
+        const int b = rem_bucket(len[r]);
+        if (b >= 0) atomicAdd(&bucket[b], 1);
+        my_work += nfull * full_chunks + rem_chunks(len[r], b);
+        my_umax = max(my_umax, max(nfull > 0 ? full_chunks : 0, rem_chunks(len[r], b)));
+      }
+      int round_total;
+      base_off[r] = written + block_exclusive_scan(nfull, warp_sums, &round_total);
+      written += round_total;
+    }
+    tot = bucket_starts(written);
+    atomicAdd(&s_work, my_work);
+    atomicMax(&s_umax, my_umax);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kPlanSpecRounds; ++r) {
+      if (r >= rounds) break;
+      const int s = r * kPlanThreads + tid;
+      const int b = s < S ? rem_bucket(len[r]) : -1;
+      pos[r] = b >= 0 ? atomicAdd(&bucket[b], 1) : -1;
+    }
+    if (waited) break;
+    wait_prerequisite_grids();                 // the kernel before has finished and its writes are visible
+    waited = true;
+    bool changed = false;
+#pragma unroll
+    for (int r = 0; r < kPlanSpecRounds; ++r) {
+      if (r >= rounds) break;
+      const int s = r * kPlanThreads + tid;
+      if (s < S && load_len(s) != len[r]) changed = true;
+    }
+    if (!__syncthreads_or(changed)) break;
+  }
+  if (tid == 0) {
+    prm.header[0] = 0;
+    prm.header[1] = (written + tot) * nt;
+    prm.header[2] = plan_working_grid(prm, tot, s_work, s_umax);
+  }
+#pragma unroll
+  for (int r = 0; r < kPlanSpecRounds; ++r) {
+    if (r >= rounds) break;
+    const int s = r * kPlanThreads + tid;
+    if (s >= S) continue;
+    const int nfull = P > 0 ? len[r] / P : 0;
+    for (int p = 0; p < nfull; ++p) prm.units[base_off[r] + p] = make_int4(s, p, 0, len[r]);
+    if (pos[r] >= 0) prm.units[pos[r]] = make_int4(s, P > 0 ? len[r] / P : 0, 0, len[r]);
   }
 }
 
@@ -1147,31 +1234,45 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    // this warp's partitions sub, sub + wph, ...: four rows in flight
-    auto row = [&](int p) { return reinterpret_cast<const float2*>(prm.part_acc + (base + p) * D + lane * PER); };
-    int p = sub;
-    for (; p + 3 * wph < np; p += 4 * wph) {
-      float2 v[4][PER / 2];
-      float w[4];
+    // this warp's partitions sub, sub + wph, ... that hold tokens, four rows
+    // in flight.  A partition with m = -inf holds none (a slot the
+    // shared-prefix kernel left empty): it is found from a ballot over the
+    // (m, l) pairs and its row is never read.
+    const unsigned share = wph == 1 ? 0xffffffffu
+                                    : (wph == 2 ? 0x55555555u : (wph == 4 ? 0x11111111u : 0x01010101u)) << sub;
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      const int pl = p0 + lane;
+      const float ml_x = pl < np ? prm.part_ml[base + pl].x : -INFINITY;
+      unsigned todo = __ballot_sync(0xffffffffu, ml_x != -INFINITY) & share;
+      while (todo) {
+        int pk[4];
+        int n = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2* src = row(p + u * wph);
+        for (int u = 0; u < 4; ++u) {
+          pk[u] = todo ? __ffs(todo) - 1 : -1;
+          if (todo) {
+            todo &= todo - 1;
+            ++n;
+          }
+        }
+        float2 v[4][PER / 2];
 #pragma unroll
-        for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
-        w[u] = prm.part_ml[base + p + u * wph].x;
+        for (int u = 0; u < 4; ++u) {
+          if (u < n) {
+            const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + pk[u]) * D + lane * PER);
+#pragma unroll
+            for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (u < n) {
+            const float wu = exp2_approx(__shfl_sync(0xffffffffu, ml_x, pk[u]) - mx);
+#pragma unroll
+            for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
+          }
+        }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float wu = exp2_approx(w[u] - mx);
-#pragma unroll
-        for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
-      }
-    }
-    for (; p < np; p += wph) {
-      const float2* src = row(p);
-      const float wu = exp2_approx(prm.part_ml[base + p].x - mx);
-#pragma unroll
-      for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), src[e]);
     }
   }
   if (wph > 1) {

@@ -309,7 +309,10 @@ pa_status launch_decode(const DecodeArgs& a) {
     rp.max_parts = np;
     rp.cap = a.max_blocks * a.BS;
     rp.part_offset = a.part_offset;
-    rp.warps_per_head = pa::reduce_warps_per_head(np);
+    // warps per head from the partitions that hold tokens: with a shared
+    // prefix, only a few of the prefix slots of a row are written (one per
+    // run of slices a prefix CTA accumulated), the rest are skipped
+    rp.warps_per_head = pa::reduce_warps_per_head(a.part_offset > 0 ? np - a.part_offset + 2 : np);
     const int heads_per_cta = pa::kReduceWarps / rp.warps_per_head;
     // programmatic dependent launch: resident early, waits for the decode grid
     cudaLaunchConfig_t cfg = {};

@@ -21,10 +21,10 @@
 
 namespace {
 
-// Split of the shared prefix into slices of this many tokens (one CTA per
-// slice, a tile of query rows and one KV head); fixed so that the workspace
-// size is a function of the arguments alone.
-constexpr int kPrefixSplitTokens = 1024;
+// Split of the shared prefix into slices of this many tokens: the units of
+// work of the prefix kernels (and the partial slots of each query row); fixed
+// so that the workspace size is a function of the arguments alone.
+constexpr int kPrefixSplitTokens = 512;
 
 int prefix_splits(int prefix_len) { return (prefix_len + kPrefixSplitTokens - 1) / kPrefixSplitTokens; }
 
@@ -40,9 +40,30 @@ bool prefix_uses_umma() {
   return !(v && std::string(v) == "mma");
 }
 
+// Queries [S][Hq][D] as a 4-D map (64 elements, D / 64 panels, Hq heads, S
+// sequences) with 128-byte swizzle, box (64, 1, G, 128 / G): one box is the
+// query-tile panel of 128 rows s * G + g of one head group.
+template <typename T>
+pa_status make_query_map(CUtensorMap* map, const void* q, int S, int Hq, int D, int G) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(Hq),
+                              static_cast<cuuint64_t>(S)};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(D) * sizeof(T),
+                                 static_cast<cuuint64_t>(Hq) * D * sizeof(T)};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(pa::kUmmaRows / G)};
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, map_type<T>(), 4, const_cast<void*>(q), dims, strides, box, elem_strides,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (queries) failed (" + std::to_string(r) + ")");
+  return PA_OK;
+}
+
 template <typename T, int D, int G>
 pa_status launch_prefix_umma(const DecodeArgs& a, const PrefixArgs& pf, const DeviceInfo& dev) {
-  int stages = 6;
+  int stages = 2;
   const int forced_st = env_int("PA_PREFIX_STAGES");
   if (forced_st >= 2 && forced_st <= 8) stages = forced_st;
   while (stages >= 2 && pa::prefix_umma_smem_bytes<D>(stages) > static_cast<size_t>(dev.smem_optin)) --stages;
@@ -57,6 +78,9 @@ pa_status launch_prefix_umma(const DecodeArgs& a, const PrefixArgs& pf, const De
   pa_status st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, 1, true, box_rows);
   if (st != PA_OK) return st;
   st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  CUtensorMap tm_q;
+  st = make_query_map<T>(&tm_q, a.q, a.S, a.Hq, D, G);
   if (st != PA_OK) return st;
   const int np = a.total_parts;
   const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
@@ -78,9 +102,14 @@ pa_status launch_prefix_umma(const DecodeArgs& a, const PrefixArgs& pf, const De
   prm.stages = stages;
   prm.stage_bytes = static_cast<uint32_t>(pa::kUmmaTile * D * sizeof(T));
   prm.qk_scale = a.scale * 1.4426950408889634f;
+  // persistent grid: one CTA per SM (it holds all the tensor memory), each
+  // taking a contiguous share of the (query-tile pair, KV head, slice) units
   constexpr int kCtaRows = pa::kUmmaTiles * pa::kUmmaRows;
-  const dim3 grid((a.S * G + kCtaRows - 1) / kCtaRows, a.Hkv, prefix_splits(pf.prefix_len));
-  kern<<<grid, pa::kUmmaThreads, smem, a.stream>>>(tm_k, tm_v, prm);
+  prm.row_pairs = (a.S * G + kCtaRows - 1) / kCtaRows;
+  prm.num_splits = prefix_splits(pf.prefix_len);
+  prm.num_units = static_cast<long long>(prm.row_pairs) * a.Hkv * prm.num_splits;
+  const int grid = prm.num_units < dev.sms ? static_cast<int>(prm.num_units) : dev.sms;
+  kern<<<grid, pa::kUmmaThreads, smem, a.stream>>>(tm_k, tm_v, tm_q, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefix_umma_kernel launch");
   return PA_OK;

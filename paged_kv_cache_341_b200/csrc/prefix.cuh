@@ -43,6 +43,9 @@ struct PrefixParams {
   int prefix_len;                // tokens, a multiple of 16
   int split_tokens;              // prefix tokens per split (multiple of kPrefixTile)
   int max_parts;                 // row stride of the partial arrays
+  int row_pairs;                 // tensor-core kernel: query-tile pairs per KV head
+  int num_splits;                // tensor-core kernel: prefix slices
+  long long num_units;           // tensor-core kernel: row_pairs x num_kv_heads x slices
   int stages;
   uint32_t stage_bytes;          // K (or V) bytes of one stage
   float qk_scale;                // scale * log2(e)

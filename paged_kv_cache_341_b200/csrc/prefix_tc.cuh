@@ -10,42 +10,46 @@
 // copy-on-write, agentechip.com "Shared Prefix Caching"), which is what the
 // tensor cores are for.
 //
-// Roles (320 threads):
-//   warp 0     TMA producer: 64-token K and V tiles of the prefix, straight
-//              from the paged cache through the block list (read once into
-//              registers), into two rings of `stages` 128-byte-swizzled tiles
-//              ([D/64 panels][64 tok][128 B]); each tile serves both query tiles.
+// Roles (576 threads):
+//   warp 0     TMA producer: both query tiles once (a 4-D box over q), then
+//              128-token K and V tiles of the prefix, straight from the paged
+//              cache through the block list (read once into registers), into
+//              two rings of `stages` 128-byte-swizzled tiles
+//              ([D/64 panels][128 tok][128 B]); each tile serves both query
+//              tiles.
 //   warp 1     allocates all 512 tensor-memory columns; lane 0 issues the
-//              MMAs.  Query tile g owns columns 256g..256g+255: S (0..63), Q
-//              (64.., D/2 columns, two 16-bit values each) and O (128..).
-//              Token tile t of query tile g:
-//                S_g(t)  = Q_g K_t^T  (M 128, N 64, K = D; A = Q from tensor
-//                                      memory, B = K from shared memory)
-//                O_g    += P_g(t) V_t (M 128, N = D, K 64; A = P from tensor
-//                                      memory where S_g(t) was)
+//              MMAs.  Query tile g owns columns 256g..256g+255: S (0..127)
+//              and O (128..).  Token tile t of query tile g:
+//                S_g(t)  = Q_g K_t^T  (M 128, N 128, K = D; both from shared memory)
+//                O_g    += P_g(t) V_t (M 128, N = D, K 128; P read from tensor
+//                                      memory over the scores: tokens 0..63 in
+//                                      S columns 0..31, 64..127 in 64..95)
 //              issued as PV_0(t), S_0(t+1), PV_1(t), S_1(t+1): while one query
 //              tile's softmax runs, the tensor core works for the other.
-//              Keeping Q in tensor memory means the only shared-memory
-//              operands are the K and V tiles themselves (2 KB per S step, 4 KB
-//              per PV step), which shared memory feeds at the full MMA rate;
-//              with Q read from shared memory as well, each S step waits on
-//              operand reads.
-//   warps 2-9  softmax of query tile (warp - 2) / 4; one query row per thread
-//              (tensor-memory lane).  First each thread writes its query row
-//              into tensor memory (tcgen05.st).  Per token tile: the 64 scores
-//              in registers, their maximum, the decode kernel's threshold rule
+//              Every MMA here is 64 cycles of tensor work (M 128, N 128,
+//              K 16); narrower tiles (N 64) were measured to take about as
+//              long per instruction, i.e. twice as long per token.
+//   warps 2-17 softmax, eight warps per query tile, two threads per query row
+//              (tensor-memory lane): thread half 0 takes scores 0..63 of a
+//              token tile, half 1 scores 64..127.  Per token tile: the
+//              maximum of each half, exchanged through shared memory between
+//              the two threads of a row; the decode kernel's threshold rule
 //              for the reference maximum (it moves only when a scaled score
-//              passes it by 2^8; O is then rescaled in tensor memory),
-//              P = 2^(s*scale*log2(e) - m) rounded to the cache's 16-bit type
-//              and stored over S as the A operand of PV; l sums the rounded
-//              weights.
+//              passes it by 2^8; each thread then rescales its half of O in
+//              tensor memory); P = 2^(s*scale*log2(e) - m) rounded to the
+//              cache's 16-bit type and stored over S as the A operand of PV;
+//              each thread sums its rounded weights, and the two sums of a
+//              row are added at the end.  Four warps per SM sub-partition
+//              share the MUFU and the other pipes, which one warp alone
+//              cannot keep busy (its instructions issue in order).
 // Products issued by one thread run in issue order, and a commit arrives only
 // once everything issued before it has completed.  So S_g(t+1) may overwrite
 // P_g(t) as soon as PV_g(t) is issued, and when S_g(t) is reported ready,
-// PV_g(t-1) has completed and O may be rescaled.  Every wait is bounded in
-// time; on a timeout all roles fall through to the end, the MMA issuer waits
-// for its own products, and the tensor memory is released before the CTA
-// exits.
+// PV_g(t-1) has completed and O may be rescaled.  Q is loaded once per CTA
+// (rows beyond the batch are zero; a second tile with no rows at all is
+// skipped).  Every wait is bounded in time; on a timeout all roles fall
+// through to the end, the MMA issuer waits for its own products, and the
+// tensor memory is released before the CTA exits.
 #ifndef PAGEDATTN_PREFIX_TC_CUH
 #define PAGEDATTN_PREFIX_TC_CUH
 
@@ -71,23 +75,75 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
+// 4-D tile load global -> shared through a tensor map, completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
+      : "memory");
+}
+
 constexpr int kUmmaRows = 128;        // query rows per tile (MMA M)
 constexpr int kUmmaTiles = 2;         // query tiles per CTA
-constexpr int kUmmaTile = 64;         // prefix tokens per stage (MMA N of S, K of PV)
-constexpr int kUmmaThreads = 64 + kUmmaTiles * 128;   // producer, MMA, softmax groups
+constexpr int kUmmaTile = 128;        // prefix tokens per stage (MMA N of S, K of PV)
+constexpr int kSoftmaxWarps = 8;                      // per query tile: two threads per row
+constexpr int kUmmaThreads = 64 + kUmmaTiles * kSoftmaxWarps * 32;   // producer, MMA, softmax groups
 constexpr uint32_t kUmmaTmemCols = 512;
-constexpr uint32_t kUmmaGroupCols = 256;              // per query tile: S 0..63, Q 64..127, O 128..255
-constexpr uint32_t kSCol = 0, kQCol = 64, kOCol = 128;
-constexpr int kGroupBars = 4;                         // mbarriers per query tile
-constexpr int kMaxSliceBlocks = 128;                  // block ids of one prefix slice held by the producer
+constexpr uint32_t kUmmaGroupCols = 256;              // per query tile: S 0..127, O 128..255
+constexpr uint32_t kSCol = 0, kOCol = 128;
+constexpr int kGroupBars = 5;                         // mbarriers per query tile
+#ifndef PA_PREFIX_POLY_EXP
+#define PA_PREFIX_POLY_EXP 2
+#endif
+// Of every 16 exponentials of the softmax, this many are evaluated on the FMA
+// pipe (exp2_poly2) and the rest by the MUFU, whose one instruction per 8
+// cycles per SM sub-partition is otherwise the softmax's bound.
+constexpr int kPolyExp = PA_PREFIX_POLY_EXP;
+static_assert(kPolyExp % 2 == 0 && kPolyExp >= 0 && kPolyExp <= 16, "pairs of exponentials");
+
+// 2^x for a pair of float32 values on the FMA pipe (no MUFU), by Cody-Waite
+// range reduction and a polynomial: x = n + f with n = round(x) and
+// |f| <= 1/2 (rounding through the float32 addition of 1.5 * 2^23), 2^f from
+// the degree-3 polynomial of least maximum relative error on [-1/2, 1/2]
+// (Remez exchange; relative error 7.5e-5, below half a unit in the last place
+// of bf16 and f16 weights), and 2^n added to the exponent field.  Inputs are
+// clamped to >= -125, so the result is a normal float32 (2^x below that is
+// returned as about 2^-125, which no weight of a row with a finite maximum
+// can tell from zero); inputs here are <= 8 (the threshold rule).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;                  // 1.5 * 2^23
+  constexpr float c0 = 0.99992807f, c1 = 0.69326099f, c2 = 0.24261112f, c3 = 0.05517167f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  float2 t = x;
+  fadd2(t, make_float2(kShift, kShift));                 // n in the low mantissa bits
+  float2 r = t;
+  fadd2(r, make_float2(-kShift, -kShift));               // n as a float, exactly
+  float2 f = x;
+  ffma2(f, r, make_float2(-1.f, -1.f));                  // f = x - n
+  float2 p = make_float2(c2, c2);
+  ffma2(p, f, make_float2(c3, c3));                      // c2 + c3 f
+  float2 p1 = make_float2(c1, c1);
+  ffma2(p1, f, p);                                       // c1 + f (c2 + c3 f)
+  float2 p0 = make_float2(c0, c0);
+  ffma2(p0, f, p1);                                      // c0 + f (...)
+  const int nx = __float_as_int(t.x) - __float_as_int(kShift);
+  const int ny = __float_as_int(t.y) - __float_as_int(kShift);
+  return make_float2(__int_as_float(__float_as_int(p0.x) + (nx << 23)),
+                     __int_as_float(__float_as_int(p0.y) + (ny << 23)));
+}
 // At least half of an SM's shared memory, so that one CTA holds the SM (and
 // all of its tensor memory) whatever the head size.
 constexpr size_t kUmmaMinSmem = 120 * 1024;
 
 template <int D>
 __host__ __device__ constexpr size_t prefix_umma_layout_bytes(int stages) {
-  return kSmemAlign + 2 * static_cast<size_t>(stages) * (D / 64) * kUmmaTile * 128      // K and V rings
-         + (4 * static_cast<size_t>(stages) + kGroupBars * kUmmaTiles + 1) * sizeof(uint64_t) + 16;
+  return kSmemAlign + kUmmaTiles * static_cast<size_t>(D / 64) * kUmmaRows * 128         // Q panels
+         + 2 * static_cast<size_t>(stages) * (D / 64) * kUmmaTile * 128                 // K and V rings
+         + (4 * static_cast<size_t>(stages) + kGroupBars * kUmmaTiles + 1 + kUmmaTiles * 4 * 3 + 1) * sizeof(uint64_t)
+         + kUmmaTiles * 2 * 3 * kUmmaRows * sizeof(float);
 }
 
 template <int D>
@@ -95,16 +151,49 @@ __host__ __device__ constexpr size_t prefix_umma_smem_bytes(int stages) {
   return prefix_umma_layout_bytes<D>(stages) < kUmmaMinSmem ? kUmmaMinSmem : prefix_umma_layout_bytes<D>(stages);
 }
 
+// Work of the persistent grid.  A unit is one slice of split_tokens prefix
+// tokens for one query-tile pair xb (rows 256 xb ..) and one KV head h;
+// units are numbered slice-fastest within a run, run = h * row_pairs + xb.
+// Each CTA takes a contiguous share of units (stream-K style), and a segment
+// is the part of its share that lies in one run: consecutive slices of the
+// same query tiles and head, accumulated into one partial (m, l, O) that goes
+// to the slot of the segment's first slice; the other slots of the segment
+// get (m, l) = (-inf, 0) and are skipped by the merge.
+struct PrefixSegment {
+  int h, split0, split1, tok_lo, tok_hi, ntiles, row0, ngroups;
+  int end;                       // first unit after the segment
+};
+
+template <int G>
+__device__ __forceinline__ PrefixSegment prefix_segment(int u, int u_end, const PrefixParams& prm) {
+  PrefixSegment Sg;
+  const int ns = prm.num_splits;
+  const int run = u / ns;
+  Sg.split0 = u - run * ns;
+  Sg.end = min(u_end, (run + 1) * ns);
+  Sg.split1 = Sg.split0 + (Sg.end - u);
+  const int xb = run % prm.row_pairs;
+  Sg.h = run / prm.row_pairs;
+  Sg.tok_lo = Sg.split0 * prm.split_tokens;
+  Sg.tok_hi = min(prm.prefix_len, Sg.split1 * prm.split_tokens);
+  Sg.ntiles = Sg.tok_hi > Sg.tok_lo ? (Sg.tok_hi - Sg.tok_lo + kUmmaTile - 1) / kUmmaTile : 0;
+  Sg.row0 = xb * (kUmmaTiles * kUmmaRows);
+  Sg.ngroups = min(kUmmaTiles, (prm.num_seqs * G - Sg.row0 + kUmmaRows - 1) / kUmmaRows);
+  return Sg;
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kUmmaThreads, 1)
     prefix_umma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       const PrefixParams prm) {
+                       const __grid_constant__ CUtensorMap tm_q, const PrefixParams prm) {
   static_assert(sizeof(T) == 2, "tensor-core path takes 16-bit caches");
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   constexpr int kHalves = D / 64;                        // 128-byte panels per row
-  constexpr uint32_t kPanel = kUmmaTile * 128;           // one panel of a K/V tile (8 KB)
+  constexpr uint32_t kPanel = kUmmaTile * 128;           // one panel of a K/V tile (16 KB)
   constexpr uint32_t kTileBytes = kHalves * kPanel;      // K (or V) bytes per stage
-  constexpr int kS = kUmmaTile;                          // scores per row and tile
+  constexpr uint32_t kQPanel = kUmmaRows * 128;          // one panel of Q (16 KB)
+  constexpr uint32_t kQBytes = kHalves * kQPanel;        // one query tile
+  constexpr int kH = 64;                                 // scores per half tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   using M = MmaType<T>;
 
@@ -112,35 +201,38 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uintptr_t base =
       (reinterpret_cast<uintptr_t>(smem) + kSmemAlign - 1) & ~static_cast<uintptr_t>(kSmemAlign - 1);
   const int stages = prm.stages;
-  unsigned char* s_k = reinterpret_cast<unsigned char*>(base);
+  unsigned char* s_q = reinterpret_cast<unsigned char*>(base);          // [tile][panel][128 rows][128 B]
+  unsigned char* s_k = s_q + kUmmaTiles * kQBytes;
   unsigned char* s_v = s_k + static_cast<size_t>(stages) * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_v + static_cast<size_t>(stages) * kTileBytes);
   uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + stages;
   uint64_t* v_full = k_empty + stages;
   uint64_t* v_empty = v_full + stages;
-  // per query tile g: s_full (S ready), p_full (P ready, O rescaled),
-  // o_done (the last PV), q_full (Q written into tensor memory)
+  // per query tile g: s_full (S ready), p_full (P ready, O rescaled), o_done
+  // (an item's last PV), o_free (the softmax has read O out), q_full (Q landed)
   uint64_t* grp = v_empty + stages;
   auto s_full = [&](int g) { return grp + kGroupBars * g; };
   auto p_full = [&](int g) { return grp + kGroupBars * g + 1; };
   auto o_done = [&](int g) { return grp + kGroupBars * g + 2; };
-  auto q_full = [&](int g) { return grp + kGroupBars * g + 3; };
+  auto o_free = [&](int g) { return grp + kGroupBars * g + 3; };
+  auto q_full = [&](int g) { return grp + kGroupBars * g + 4; };
   uint64_t* drain = grp + kGroupBars * kUmmaTiles;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  // the two threads of a row exchange their halves' maxima (per query tile,
+  // lane quarter and token-tile parity) and, at the end of an item, their sums
+  uint64_t* pair_bars = drain + 1;                      // [tile][quarter][parity]
+  uint64_t* sum_bars = pair_bars + kUmmaTiles * 4 * 2;  // [tile][quarter]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sum_bars + kUmmaTiles * 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // row maxima of the two score halves, [tile][half][tile parity][row], then sums [tile][half][row]
+  float* s_xmax = reinterpret_cast<float*>(sum_bars + kUmmaTiles * 4 + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int split = blockIdx.z;
-  const int tok_lo = split * prm.split_tokens;
-  const int tok_hi = min(prm.prefix_len, tok_lo + prm.split_tokens);
-  const int ntiles = tok_hi > tok_lo ? (tok_hi - tok_lo + kUmmaTile - 1) / kUmmaTile : 0;
   const int rows_total = prm.num_seqs * G;
-  const int row0 = blockIdx.x * (kUmmaTiles * kUmmaRows);
-  // query tiles of this CTA that hold at least one row
-  const int ngroups = min(kUmmaTiles, (rows_total - row0 + kUmmaRows - 1) / kUmmaRows);
+  // this CTA's share of the units
+  const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * prm.num_units / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * prm.num_units / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < stages; ++i) {
@@ -152,11 +244,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // softmax-side barriers take one arrival per warp (elected lane after __syncwarp)
     for (int g = 0; g < kUmmaTiles; ++g) {
       mbar_init(s_full(g), 1);
-      mbar_init(p_full(g), 4);
+      mbar_init(p_full(g), kSoftmaxWarps);
       mbar_init(o_done(g), 1);
-      mbar_init(q_full(g), 4);
+      mbar_init(o_free(g), kSoftmaxWarps);
+      mbar_init(q_full(g), 1);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kUmmaTiles * 4 * 3; ++i) mbar_init(&pair_bars[i], 2);   // pair and sum barriers
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,78 +272,82 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const uint64_t policy = policy_evict_last();
     const int BS = prm.block_size;
     const int piece_rows = BS < kChunkTokens ? BS : kChunkTokens;
-    // the slice's block ids, read once: lane i holds entries i, i + 32, ...
-    // (a slice of split_tokens <= 1024 tokens spans at most 128 blocks of 8)
-    const int blk_lo = tok_lo / BS;
-    const int nblk = tok_hi > tok_lo ? (tok_hi - 1) / BS - blk_lo + 1 : 0;
-    int ids[kMaxSliceBlocks / 32];
-#pragma unroll
-    for (int k = 0; k < kMaxSliceBlocks / 32; ++k) {
-      const int b = lane + 32 * k;
-      ids[k] = b < nblk ? prm.prefix_blocks[blk_lo + b] : 0;
-    }
     int kst = 0, vst = 0;
     uint32_t kph = 0, vph = 0;
     int k_armed = 0, v_armed = 0;     // tiles whose K (V) copies were issued
-    for (int t = 0; t < ntiles; ++t) {
-      const int tok0 = tok_lo + t * kUmmaTile;
-      const int ntok = min(kUmmaTile, tok_hi - tok0);
-      const int npieces = ntok / piece_rows;     // <= 8
-      // one box per lane: piece pc = lane / kHalves, panel hf = lane % kHalves
-      const int nbox = npieces * kHalves;        // <= 16
-      const int pc = lane / kHalves;
-      const int hf = lane - pc * kHalves;
-      const int tk = tok0 + (lane < nbox ? pc : 0) * piece_rows;
-      const int bl = tk / BS - blk_lo;           // entry of this lane's piece in the slice
-      int phys = 0;
-#pragma unroll
-      for (int k = 0; k < kMaxSliceBlocks / 32; ++k) {
-        const int v = __shfl_sync(0xffffffffu, ids[k], bl & 31);
-        if ((bl >> 5) == k) phys = v;
-      }
-      int row = 0;
-      if (lane < nbox) {
-        if (phys < 0 || phys >= prm.num_blocks) {
-          set_device_error(DEVERR_BAD_BLOCK_ID);
-          phys = 0;
+    bool ok = true;
+    for (int u = u_begin; ok && u < u_end;) {
+      const PrefixSegment I = prefix_segment<G>(u, u_end, prm);
+      u = I.end;
+      // the block id of this lane's piece of each tile, read one tile ahead
+      auto piece_block = [&](int t) {
+        const int tok0 = I.tok_lo + t * kUmmaTile;
+        const int ntok = min(kUmmaTile, I.tok_hi - tok0);
+        const int pc = lane / kHalves;
+        return pc * piece_rows < ntok ? __ldg(prm.prefix_blocks + (tok0 + pc * piece_rows) / BS) : 0;
+      };
+      int next_phys = I.ntiles > 0 ? piece_block(0) : 0;
+      for (int t = 0; t < I.ntiles; ++t) {
+        const int tok0 = I.tok_lo + t * kUmmaTile;
+        const int ntok = min(kUmmaTile, I.tok_hi - tok0);
+        const int npieces = ntok / piece_rows;     // <= 16
+        // one box per lane: piece pc = lane / kHalves, panel hf = lane % kHalves
+        const int nbox = npieces * kHalves;        // <= 32
+        const int pc = lane / kHalves;
+        const int hf = lane - pc * kHalves;
+        int phys = next_phys;
+        if (t + 1 < I.ntiles) next_phys = piece_block(t + 1);
+        int row = 0;
+        if (lane < nbox) {
+          if (phys < 0 || phys >= prm.num_blocks) {
+            set_device_error(DEVERR_BAD_BLOCK_ID);
+            phys = 0;
+          }
+          const int tk = tok0 + pc * piece_rows;
+          row = phys * BS + (tk - (tk / BS) * BS);
         }
-        row = phys * BS + (tk - (bl + blk_lo) * BS);
-      }
-      const uint32_t tx = static_cast<uint32_t>(nbox) * piece_rows * 128;
-      // K tile
-      if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[kst], kph ^ 1, abort_flag))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&k_full[kst], tx);
-      __syncwarp();
-      if (lane < nbox)
-        tma_load_3d(s_k + static_cast<size_t>(kst) * kTileBytes + hf * kPanel + pc * piece_rows * 128, &tm_k,
-                    &k_full[kst], 0, h * kHalves + hf, row, policy);
-      ++k_armed;
-      if (++kst == stages) {
-        kst = 0;
-        kph ^= 1;
-      }
-      // V tile; rows past the end of a short last tile are zeroed so that
-      // P = 0 there never meets stale bits
-      if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[vst], vph ^ 1, abort_flag))) break;
-      unsigned char* vdst = s_v + static_cast<size_t>(vst) * kTileBytes;
-      if (ntok < kUmmaTile) {
-        const int chunks = (kUmmaTile - ntok) * 8;     // 16-byte chunks per panel
-        for (int i = lane; i < kHalves * chunks; i += 32) {
-          const int p = i / chunks, c = i - p * chunks;
-          *reinterpret_cast<uint4*>(vdst + p * kPanel + ntok * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        const uint32_t tx = static_cast<uint32_t>(nbox) * piece_rows * 128;
+        // K tile
+        if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[kst], kph ^ 1, abort_flag))) {
+          ok = false;
+          break;
         }
-        tc::fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&v_full[vst], tx);
-      __syncwarp();
-      if (lane < nbox)
-        tma_load_3d(vdst + hf * kPanel + pc * piece_rows * 128, &tm_v, &v_full[vst], 0, h * kHalves + hf, row,
-                    policy);
-      ++v_armed;
-      if (++vst == stages) {
-        vst = 0;
-        vph ^= 1;
+        if (lane == 0) mbar_arrive_expect_tx(&k_full[kst], tx);
+        __syncwarp();
+        if (lane < nbox)
+          tma_load_3d(s_k + static_cast<size_t>(kst) * kTileBytes + hf * kPanel + pc * piece_rows * 128, &tm_k,
+                      &k_full[kst], 0, I.h * kHalves + hf, row, policy);
+        ++k_armed;
+        if (++kst == stages) {
+          kst = 0;
+          kph ^= 1;
+        }
+        // V tile; rows past the end of a short last tile are zeroed so that
+        // P = 0 there never meets stale bits
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[vst], vph ^ 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        unsigned char* vdst = s_v + static_cast<size_t>(vst) * kTileBytes;
+        if (ntok < kUmmaTile) {
+          const int chunks = (kUmmaTile - ntok) * 8;     // 16-byte chunks per panel
+          for (int i = lane; i < kHalves * chunks; i += 32) {
+            const int p = i / chunks, c = i - p * chunks;
+            *reinterpret_cast<uint4*>(vdst + p * kPanel + ntok * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+          tc::fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&v_full[vst], tx);
+        __syncwarp();
+        if (lane < nbox)
+          tma_load_3d(vdst + hf * kPanel + pc * piece_rows * 128, &tm_v, &v_full[vst], 0, I.h * kHalves + hf, row,
+                      policy);
+        ++v_armed;
+        if (++vst == stages) {
+          vst = 0;
+          vph ^= 1;
+        }
       }
     }
     // copies still in flight must land before the CTA may exit
@@ -282,246 +380,315 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       // descriptors of the operand bases; an operand at byte offset x from a
       // base is the base descriptor plus x >> 4 (start-address field, no carry
       // below 256 KB of shared memory)
+      const uint64_t q_desc = tc::smem_desc_sw128(smem_addr(s_q), 16, 1024);
       const uint64_t k_desc = tc::smem_desc_sw128(smem_addr(s_k), 16, 1024);
       const uint64_t v_desc = tc::smem_desc_sw128(smem_addr(s_v), kPanel, 1024);
       bool ok = true;
-      for (int g = 0; g < ngroups && ok; ++g) ok = mbar_wait(q_full(g), 0, abort_flag);
-      tc::fence_after_sync();
       int kst = 0, vst = 0;
       uint32_t kph = 0, vph = 0;
-      // S_g = Q_g K^T (Q in tensor memory, 8 columns per K = 16 step)
+      int items_g[kUmmaTiles] = {0, 0};          // items each query tile has taken so far
+      int tiles_g[kUmmaTiles] = {0, 0};          // token tiles each query tile has taken so far
+      // S_g = Q_g K^T into columns 256g..256g+127
       auto issue_s = [&](int g, int ks) {
         const uint64_t kb = k_desc + ((ks * kTileBytes) >> 4);
-        const uint32_t col = tmem + g * kUmmaGroupCols;
+        const uint64_t qb = q_desc + ((g * kQBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          tc::mma_f16_ts(col + kSCol, col + kQCol + kk * 8, kb + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4),
-                         idesc_s, kk > 0);
+          tc::mma_f16_ss(tmem + g * kUmmaGroupCols + kSCol, qb + (((kk >> 2) * kQPanel + (kk & 3) * 32) >> 4),
+                         kb + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
         tc::commit(s_full(g));
       };
-      // O_g += P_g V; P in the first 32 columns of S, two 16-bit values per column
+      // O_g += P_g V; P two 16-bit values per column, tokens 0..63 in S
+      // columns 0..31 and tokens 64..127 in S columns 64..95 (each softmax
+      // thread writes its weights over its own half of the scores)
       auto issue_pv = [&](int g, int vs, bool first) {
         const uint64_t vb = v_desc + ((vs * kTileBytes) >> 4);
         const uint32_t col = tmem + g * kUmmaGroupCols;
 #pragma unroll
         for (int kk = 0; kk < kUmmaTile / 16; ++kk)
-          tc::mma_f16_ts(col + kOCol, col + kSCol + kk * 8, vb + ((kk * 16 * 128) >> 4), idesc_o, !first || kk > 0);
+          tc::mma_f16_ts(col + kOCol, col + kSCol + kk * 8 + (kk >= 4 ? 32 : 0), vb + ((kk * 16 * 128) >> 4), idesc_o,
+                         !first || kk > 0);
       };
-      if (ok && ntiles > 0) {
-        ok = mbar_wait(&k_full[kst], kph, abort_flag);
-        if (ok) {
-          tc::fence_after_sync();
-          for (int g = 0; g < ngroups; ++g) issue_s(g, kst);
-          tc::commit(&k_empty[kst]);
-          if (++kst == stages) {
-            kst = 0;
-            kph ^= 1;
-          }
-        }
-      }
-      for (int t = 0; ok && t < ntiles; ++t) {
-        const bool more = t + 1 < ntiles;
-        if (!mbar_wait(&v_full[vst], vph, abort_flag)) {
-          ok = false;
-          break;
-        }
-        for (int g = 0; g < ngroups; ++g) {
-          // P_g(t) written (and O rescaled if the maximum moved)
-          if (!mbar_wait(p_full(g), t & 1, abort_flag)) {
+      for (int u = u_begin; ok && u < u_end;) {
+        const PrefixSegment I = prefix_segment<G>(u, u_end, prm);
+        u = I.end;
+        for (int g = 0; g < I.ngroups && ok; ++g) ok = mbar_wait(q_full(g), items_g[g] & 1, abort_flag);
+        if (!ok) break;
+        tc::fence_after_sync();
+        if (I.ntiles > 0) {
+          if (!mbar_wait(&k_full[kst], kph, abort_flag)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          issue_pv(g, vst, t == 0);
-          if (more) {
-            if (g == 0) {
-              if (!mbar_wait(&k_full[kst], kph, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc::fence_after_sync();
-            }
-            issue_s(g, kst);                         // overwrites P_g(t) after PV_g(t) in issue order
-          }
-        }
-        if (!ok) break;
-        tc::commit(&v_empty[vst]);
-        if (++vst == stages) {
-          vst = 0;
-          vph ^= 1;
-        }
-        if (more) {
+          for (int g = 0; g < I.ngroups; ++g) issue_s(g, kst);
           tc::commit(&k_empty[kst]);
           if (++kst == stages) {
             kst = 0;
             kph ^= 1;
           }
         }
+        for (int t = 0; ok && t < I.ntiles; ++t) {
+          const bool more = t + 1 < I.ntiles;
+          if (!mbar_wait(&v_full[vst], vph, abort_flag) || (more && !mbar_wait(&k_full[kst], kph, abort_flag))) {
+            ok = false;
+            break;
+          }
+          for (int g = 0; g < I.ngroups; ++g) {
+            // P_g(t) written (and O rescaled if the maximum moved); before the
+            // first product of an item, the previous item's O read out
+            if (!mbar_wait(p_full(g), tiles_g[g] & 1, abort_flag) ||
+                (t == 0 && items_g[g] > 0 && !mbar_wait(o_free(g), (items_g[g] - 1) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            ++tiles_g[g];
+            tc::fence_after_sync();
+            issue_pv(g, vst, t == 0);
+            if (more) issue_s(g, kst);                // overwrites P_g(t) after PV_g(t) in issue order
+          }
+          if (!ok) break;
+          tc::commit(&v_empty[vst]);
+          if (++vst == stages) {
+            vst = 0;
+            vph ^= 1;
+          }
+          if (more) {
+            tc::commit(&k_empty[kst]);
+            if (++kst == stages) {
+              kst = 0;
+              kph ^= 1;
+            }
+          }
+        }
+        if (!ok) break;
+        for (int g = 0; g < I.ngroups; ++g) {
+          tc::commit(o_done(g));
+          ++items_g[g];
+        }
       }
-      for (int g = 0; g < ngroups; ++g) tc::commit(o_done(g));
       // every product issued above completes before the tensor memory goes
       tc::commit(drain);
       mbar_wait_drain(drain, 0);
     }
     __syncwarp();
-  } else if ((warp - 2) / 4 < ngroups) {
+  } else {
     // ------------------------------------------------------------- softmax
-    const int g = (warp - 2) / 4;                              // query tile of this group
+    const int g = (warp - 2) / kSoftmaxWarps;                  // query tile of this group
+    const int half = ((warp - 2) % kSoftmaxWarps) / 4;         // scores 64 * half .. 64 * half + 63
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;                       // tensor-memory lane = query row in the tile
     const uint32_t t_lane = tmem + g * kUmmaGroupCols + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int gr = row0 + g * kUmmaRows + row;
-    const bool valid = gr < rows_total;
-    const int s_idx = valid ? gr / G : 0;
-    const int g_idx = valid ? gr - s_idx * G : 0;
+    const bool leader = (warp - 2) % kSoftmaxWarps == 0 && lane == 0;   // loads this group's query tiles
     const float qk = prm.qk_scale;
     const float pad = qk >= 0.f ? -INFINITY : INFINITY;
     const float2 qk2 = make_float2(qk, qk);
-    float m = -INFINITY, l = 0.f;
-
-    // this thread's query row into tensor memory (zeros past the batch):
-    // element 2c in the low half of column kQCol + c
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(prm.q) +
-                                                        (static_cast<size_t>(s_idx) * prm.num_q_heads + h * G + g_idx) * D);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t qr[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = valid ? __ldg(src + c * 8 + i) : make_uint4(0, 0, 0, 0);
-          qr[4 * i] = v.x;
-          qr[4 * i + 1] = v.y;
-          qr[4 * i + 2] = v.z;
-          qr[4 * i + 3] = v.w;
-        }
-        tc::tmem_st32(t_lane + kQCol + c * 32, qr);
+    // the two warps holding this lane quarter's rows meet at these barriers
+    // (one arrival per warp; waits bounded like every other)
+    uint64_t* pair_bar = pair_bars + (g * 4 + quarter) * 2;   // + tile parity
+    uint64_t* sum_bar = sum_bars + g * 4 + quarter;
+    float* x_max = s_xmax + (g * 2 + half) * 2 * kUmmaRows;              // [tile parity][row], own half
+    const float* y_max = s_xmax + (g * 2 + (half ^ 1)) * 2 * kUmmaRows;  // the other half
+    float* s_sum = s_xmax + kUmmaTiles * 2 * 2 * kUmmaRows;              // [tile][half][row]
+    // the first unit, from `u` on, of a segment in which this query tile takes
+    // part (u_end if none)
+    auto next_segment = [&](int u) {
+      while (u < u_end) {
+        const PrefixSegment J = prefix_segment<G>(u, u_end, prm);
+        if (g < J.ngroups) return u;
+        u = J.end;
       }
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_full(g));
+      return u_end;
+    };
+    // the query tile g of the segment starting at unit u into shared memory:
+    // the box (64 elements, G heads, 128 / G sequences) of q viewed as
+    // [S][Hq][D / 64 panels][64]; rows past the batch read as zeros
+    auto load_q = [&](int u) {
+      const PrefixSegment J = prefix_segment<G>(u, u_end, prm);
+      mbar_arrive_expect_tx(q_full(g), kQBytes);
+      for (int hf = 0; hf < kHalves; ++hf)
+        tma_load_4d(s_q + g * kQBytes + hf * kQPanel, &tm_q, q_full(g), 0, hf, J.h * G, (J.row0 + g * kUmmaRows) / G);
+    };
+    const int first = next_segment(u_begin);
+    if (leader) {
+      prefetch_tensormap(&tm_q);
+      if (first < u_end) load_q(first);
     }
-
+    int tiles = 0;                               // token tiles this query tile has taken so far
+    int items = 0;                               // segments this query tile has taken so far
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
-      const int ntok = min(kUmmaTile, tok_hi - (tok_lo + t * kUmmaTile));
-      const bool full = ntok == kUmmaTile;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), t & 1, abort_flag))) {
+    for (int u = first; ok && u < u_end;) {
+      const PrefixSegment I = prefix_segment<G>(u, u_end, prm);
+      u = next_segment(I.end);
+      const int gr = I.row0 + g * kUmmaRows + row;
+      const bool valid = gr < rows_total;
+      const int s_idx = valid ? gr / G : 0;
+      const int g_idx = valid ? gr - s_idx * G : 0;
+      float m = -INFINITY, l = 0.f;
+      for (int t = 0; t < I.ntiles; ++t, ++tiles) {
+        const int ntok = min(kUmmaTile, I.tok_hi - (I.tok_lo + t * kUmmaTile));
+        const int nh = min(kH, max(0, ntok - half * kH));         // valid scores in this half
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full(g), tiles & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        // the segment's last S has completed, so its query tile may be replaced
+        if (t == I.ntiles - 1 && leader && u < u_end) load_q(u);
+        const uint32_t s_col = t_lane + kSCol + half * kH;
+        // maximum (minimum for a negative scale) of this half's raw scores, 32 at a time
+        float ext = pad;
+#pragma unroll
+        for (int q32 = 0; q32 < 2; ++q32) {
+          uint32_t x[32];
+          tc::tmem_ld32(s_col + q32 * 32, x);
+          tc::tmem_wait_ld();
+          if (nh < kH) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = q32 * 32 + j < nh ? x[j] : __float_as_uint(pad);
+          }
+          float cm[4] = {__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]), __uint_as_float(x[3])};
+          if (qk >= 0.f) {
+#pragma unroll
+            for (int j = 4; j < 28; j += 8)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) cm[k] = fmax3(cm[k], __uint_as_float(x[j + k]), __uint_as_float(x[j + 4 + k]));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __uint_as_float(x[28 + k]));
+            ext = fmax3(ext, fmax3(cm[0], cm[1], cm[2]), cm[3]);
+          } else {
+#pragma unroll
+            for (int j = 4; j < 28; j += 8)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) cm[k] = fmin3(cm[k], __uint_as_float(x[j + k]), __uint_as_float(x[j + 4 + k]));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cm[k] = fminf(cm[k], __uint_as_float(x[28 + k]));
+            ext = fmin3(ext, fmin3(cm[0], cm[1], cm[2]), cm[3]);
+          }
+        }
+        // the row's scaled maximum: this half's and the other thread's
+        const float c_own = nh > 0 ? ext * qk : -INFINITY;
+        x_max[(tiles & 1) * kUmmaRows + row] = c_own;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pair_bar[tiles & 1]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&pair_bar[tiles & 1], (tiles >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const float c = fmaxf(c_own, y_max[(tiles & 1) * kUmmaRows + row]);
+        if (__any_sync(0xffffffffu, c > m + kTau)) {
+          const float mn = c > m + kTau ? c : m;
+          const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
+          if (t >= 1) {
+            // O holds PV(0..t-1) of this item, all completed (S(t) was issued
+            // after PV(t-1)); PV(t) waits for this tile's P.  This thread's half of O.
+#pragma unroll 1
+            for (int ob = 0; ob < D / 32; ++ob) {
+              uint32_t o[16];
+              tc::tmem_ld16(t_lane + kOCol + half * (D / 2) + ob * 16, o);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+              tc::tmem_st16(t_lane + kOCol + half * (D / 2) + ob * 16, o);
+            }
+          }
+          l *= f;
+          m = mn;
+        }
+        // P = 2^(s * qk - m), rounded to T, two per column: tokens 64 * half + j
+        // go to column 64 * half + j / 2, i.e. over this thread's own scores
+        // already read (the other thread's columns are never touched).  Of
+        // every 16 exponentials, kPolyExp are taken by the FMA-pipe polynomial.
+        const float2 nm2 = make_float2(-m, -m);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int q32 = 0; q32 < 2; ++q32) {
+          uint32_t x[32];
+          tc::tmem_ld32(s_col + q32 * 32, x);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float2 e = nm2;
+            ffma2(e, make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), qk2);
+            x[2 * i] = __float_as_uint(e.x);
+            x[2 * i + 1] = __float_as_uint(e.y);
+          }
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+#pragma unroll
+            for (int j = 0; j < 16 - kPolyExp; ++j)
+              x[16 * b + j] = __float_as_uint(exp2_approx(__uint_as_float(x[16 * b + j])));
+#pragma unroll
+            for (int j = 16 - kPolyExp; j < 16; j += 2) {
+              const float2 y =
+                  exp2_poly2(make_float2(__uint_as_float(x[16 * b + j]), __uint_as_float(x[16 * b + j + 1])));
+              x[16 * b + j] = __float_as_uint(y.x);
+              x[16 * b + j + 1] = __float_as_uint(y.y);
+            }
+          }
+          if (nh < kH) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = q32 * 32 + j < nh ? x[j] : 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            w[i] = M::pack(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+            fadd2(ls[i & 1], M::unpack(w[i]));
+          }
+          tc::tmem_st16(t_lane + kSCol + half * kH + q32 * 16, w);
+        }
+        tc::tmem_wait_st();
+        l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(g));
+      }
+      if (!ok) break;
+      if (I.ntiles > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done(g), items & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      uint32_t cur[kS];
-      tc::tmem_ld32_at<0>(t_lane + kSCol, cur);
-      tc::tmem_ld32_at<32>(t_lane + kSCol + 32, cur);
-      tc::tmem_wait_ld();
-      if (!full) {
-#pragma unroll
-        for (int j = 0; j < kS; ++j) cur[j] = j < ntok ? cur[j] : __float_as_uint(pad);
+      // the row sum: this half's and the other thread's
+      s_sum[(g * 2 + half) * kUmmaRows + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sum_bar);
+      if (!__all_sync(0xffffffffu, mbar_wait(sum_bar, items & 1, abort_flag))) {
+        ok = false;
+        break;
       }
-      // maximum (minimum for a negative scale) of the raw scores: four
-      // chains of three-input max over the 64 scores
-      float cm[4];
+      const float l_row = l + s_sum[(g * 2 + (half ^ 1)) * kUmmaRows + row];
+      const size_t pi = (static_cast<size_t>(s_idx) * prm.num_q_heads + I.h * G + g_idx) * prm.max_parts + I.split0;
+      float* dst = prm.part_acc + pi * D + half * (D / 2);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cm[i] = __uint_as_float(cur[i]);
-      float ext;
-      if (qk >= 0.f) {
+      for (int cb = 0; cb < D / 64; ++cb) {
+        uint32_t o[32];
+        if (I.ntiles > 0) {
+          tc::tmem_ld32(t_lane + kOCol + half * (D / 2) + cb * 32, o);
+          tc::tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int j = 4; j < kS - 4; j += 8)
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        if (valid) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) cm[k] = fmax3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __uint_as_float(cur[kS - 4 + k]));
-        ext = fmax3(fmaxf(cm[0], cm[1]), cm[2], cm[3]);
-      } else {
-#pragma unroll
-        for (int j = 4; j < kS - 4; j += 8)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) cm[k] = fmin3(cm[k], __uint_as_float(cur[j + k]), __uint_as_float(cur[j + 4 + k]));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cm[k] = fminf(cm[k], __uint_as_float(cur[kS - 4 + k]));
-        ext = fmin3(fminf(cm[0], cm[1]), cm[2], cm[3]);
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + cb * 32 + j) =
+                make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
+                            __uint_as_float(o[j + 3]));
+        }
       }
-      const float c = ext * qk;
-      if (__any_sync(0xffffffffu, c > m + kTau)) {
-        const float mn = c > m + kTau ? c : m;
-        const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
-        if (t >= 1) {
-          // O holds PV(0..t-1), all completed (S(t) was issued after PV(t-1));
-          // PV(t) waits for this tile's P
-#pragma unroll 1
-          for (int ob = 0; ob < D / 16; ++ob) {
-            uint32_t o[16];
-            tc::tmem_ld16(t_lane + kOCol + ob * 16, o);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-            tc::tmem_st16(t_lane + kOCol + ob * 16, o);
-          }
-        }
-        l *= f;
-        m = mn;
+      if (valid && half == 0) {
+        prm.part_ml[pi] = make_float2(m, l_row);
+        for (int sp = 1; sp < I.split1 - I.split0; ++sp) prm.part_ml[pi + sp] = make_float2(-INFINITY, 0.f);
       }
-      // P = 2^(s * qk - m), rounded to T, two per column over this tile's S;
-      // the row sum takes the rounded values.  Three sweeps per half of the
-      // scores (exponents, exponentials, packing), so the 32 exponentials are
-      // independent and stream through the MUFU.
-      const float2 nm2 = make_float2(-m, -m);
-      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t* x = cur + half * 32;           // the scores become exponents, then weights, in place
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float2 e = nm2;
-          ffma2(e, make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), qk2);
-          x[2 * i] = __float_as_uint(e.x);
-          x[2 * i + 1] = __float_as_uint(e.y);
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(exp2_approx(__uint_as_float(x[j])));
-        if (!full) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = half * 32 + j < ntok ? x[j] : 0u;
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          w[i] = M::pack(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
-          fadd2(ls[i & 1], M::unpack(w[i]));
-        }
-        tc::tmem_st16(t_lane + kSCol + half * 16, w);
-      }
-      tc::tmem_wait_st();
-      l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
+      // O has been read out: the next item's first product may overwrite it
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(g));
+      if (lane == 0) mbar_arrive(o_free(g));
+      ++items;
     }
-    if (ok && ntiles > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done(g), 0, abort_flag))) ok = false;
-    tc::fence_after_sync();
-    const size_t pi = (static_cast<size_t>(s_idx) * prm.num_q_heads + h * G + g_idx) * prm.max_parts + split;
-    float* dst = prm.part_acc + pi * D;
-#pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
-      uint32_t o[32];
-      if (ok && ntiles > 0) {
-        tc::tmem_ld32(t_lane + kOCol + cb * 32, o);
-        tc::tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = 0u;
-      }
-      if (valid && ok) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + cb * 32 + j) =
-              make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]), __uint_as_float(o[j + 2]),
-                          __uint_as_float(o[j + 3]));
-      }
-    }
-    if (valid && ok) prm.part_ml[pi] = make_float2(m, l);
   }
 
   tc::fence_before_sync();
