@@ -153,7 +153,11 @@ __host__ __device__ constexpr size_t prefix_umma_smem_bytes(int stages) {
 
 // Work of the persistent grid.  A unit is one slice of split_tokens prefix
 // tokens for one query-tile pair xb (rows 256 xb ..) and one KV head h;
-// units are numbered slice-fastest within a run, run = h * row_pairs + xb.
+// units are numbered slice-fastest within a run, run = xb * num_kv_heads + h.
+// With the query-tile pairs outermost, equal shares put the CTAs that need the
+// same (head, slice) for different query tiles at the same slice at the same
+// time whenever the grid is a multiple of the number of pairs (148 CTAs and 4
+// pairs here), so each K/V tile comes from DRAM once and from L2 after.
 // Each CTA takes a contiguous share of units (stream-K style), and a segment
 // is the part of its share that lies in one run: consecutive slices of the
 // same query tiles and head, accumulated into one partial (m, l, O) that goes
@@ -172,8 +176,8 @@ __device__ __forceinline__ PrefixSegment prefix_segment(int u, int u_end, const 
   Sg.split0 = u - run * ns;
   Sg.end = min(u_end, (run + 1) * ns);
   Sg.split1 = Sg.split0 + (Sg.end - u);
-  const int xb = run % prm.row_pairs;
-  Sg.h = run / prm.row_pairs;
+  const int xb = run / prm.num_kv_heads;
+  Sg.h = run - xb * prm.num_kv_heads;
   Sg.tok_lo = Sg.split0 * prm.split_tokens;
   Sg.tok_hi = min(prm.prefix_len, Sg.split1 * prm.split_tokens);
   Sg.ntiles = Sg.tok_hi > Sg.tok_lo ? (Sg.tok_hi - Sg.tok_lo + kUmmaTile - 1) / kUmmaTile : 0;
