@@ -1223,17 +1223,27 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
   float mx = -INFINITY, lsum = 0.f;
   if (active) {
-    // every warp of the head computes M and L over all partitions (np (m, l) pairs)
-    for (int p = lane; p < np; p += 32) mx = fmaxf(mx, prm.part_ml[base + p].x);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
+    // every warp of the head computes M and L over all partitions in one
+    // sweep of the (m, l) pairs: each lane keeps a running maximum and a sum
+    // rescaled to it, and the lanes' pairs are merged the same way
     for (int p = lane; p < np; p += 32) {
       const float2 ml = prm.part_ml[base + p];
-      lsum += ml.y * exp2_approx(ml.x - mx);
+      if (ml.x > mx) {
+        lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
+        mx = ml.x;
+      } else if (ml.x != -INFINITY) {
+        lsum += ml.y * exp2_approx(ml.x - mx);
+      }
     }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
+      const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
+      const float mn = fmaxf(mx, mo);
+      lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) + (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
+      mx = mn;
+    }
+    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
     // this warp's partitions sub, sub + wph, ... that hold tokens, four rows
     // in flight.  A partition with m = -inf holds none (a slot the
     // shared-prefix kernel left empty): it is found from a ballot over the

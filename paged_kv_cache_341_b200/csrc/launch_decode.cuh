@@ -176,10 +176,13 @@ pa_status launch_decode(const DecodeArgs& a) {
 
   // Launch shape, chosen by measurement on B200 (sweep over 1/2/4/8 KV heads
   // per CTA x 2..6 stages on the four large workloads): one KV head per CTA
-  // and a 3-deep ring, i.e. small CTAs, about seven per SM, whose independent
+  // and a 2- or 3-deep ring, i.e. small CTAs, eight per SM, whose independent
   // producers keep HBM busy, beat fewer, wider CTAs by up to 25%.
   int ht = 1;
-  int stages = 3;
+  // 3 stages for groups up to 4; 2 for 8 query heads per KV head, whose
+  // consumer spends longer on each stage (70B-shaped call: 5,569 -> 5,653 GB/s,
+  // while the Llama shapes lose 2 % with 2)
+  int stages = G >= 8 ? 2 : 3;
   const int forced_ht = env_int("PA_DECODE_TILE_HEADS");
   if (forced_ht > 0 && forced_ht <= pa::kMaxTileHeads && a.Hkv % forced_ht == 0) ht = forced_ht;
   const int forced_st = env_int("PA_DECODE_STAGES");
