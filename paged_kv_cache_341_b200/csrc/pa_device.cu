@@ -14,6 +14,7 @@
 #include "decode.cuh"
 #include "prefix.cuh"
 #include "prefix_tc.cuh"
+#include "prefix_tc2.cuh"
 #include "pa.h"
 #include "pa_common.h"
 
@@ -33,11 +34,17 @@ struct PrefixArgs {
   int prefix_len;
 };
 
-// Prefix kernel: tcgen05 (tensor memory) by default; PA_PREFIX_PATH=mma picks
-// the mma.sync kernel (same results within rounding, kept for comparison).
-bool prefix_uses_umma() {
+// Prefix kernel: the one-SM tcgen05 kernel by default; PA_PREFIX_PATH=pair
+// picks the SM-pair tcgen05 kernel (head_dim 128, where clusters of two fit;
+// else the default) and PA_PREFIX_PATH=mma the mma.sync kernel (same results
+// within rounding, kept for comparison).
+enum class PrefixPath { kUmma, kPair, kMma };
+thread_local int g_last_prefix_kernel = 0;     // pa_debug_last_prefix_kernel
+PrefixPath prefix_path() {
   const char* v = std::getenv("PA_PREFIX_PATH");
-  return !(v && std::string(v) == "mma");
+  if (v && std::string(v) == "mma") return PrefixPath::kMma;
+  if (v && std::string(v) == "pair") return PrefixPath::kPair;
+  return PrefixPath::kUmma;
 }
 
 // Queries [S][Hq][D] as a 4-D map (64 elements, D / 64 panels, Hq heads, S
@@ -112,6 +119,99 @@ pa_status launch_prefix_umma(const DecodeArgs& a, const PrefixArgs& pf, const De
   kern<<<grid, pa::kUmmaThreads, smem, a.stream>>>(tm_k, tm_v, tm_q, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefix_umma_kernel launch");
+  g_last_prefix_kernel = 2;
+  return PA_OK;
+}
+
+// The SM-pair kernel (head_dim 128): clusters of two CTAs, as many as can be
+// resident at once.  Returns PA_ERR_UNSUPPORTED without launching when no
+// cluster of two fits, and the caller falls back to the one-SM kernel.
+template <typename T, int G>
+pa_status launch_prefix_pair(const DecodeArgs& a, const PrefixArgs& pf, const DeviceInfo& dev) {
+  constexpr int D = 128;
+  int stages = 4;
+  const int forced_st = env_int("PA_PREFIX_STAGES");
+  if (forced_st >= 2 && forced_st <= 8) stages = forced_st;
+  while (stages >= 2 && pa::prefix_pair_smem_bytes<D>(stages) > static_cast<size_t>(dev.smem_optin)) --stages;
+  if (stages < 2) return PA_ERR_UNSUPPORTED;
+  const size_t smem = pa::prefix_pair_smem_bytes<D>(stages);
+  auto kern = pa::prefix_pair_kernel<T, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix pair)");
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(pa::kPairThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = a.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // resident clusters of two for this kernel and size, once per device
+  static std::mutex mu;
+  static int max_clusters[64][9] = {};
+  int dev_id = 0;
+  e = cudaGetDevice(&dev_id);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int resident = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    int& slot = max_clusters[dev_id < 64 ? dev_id : 63][stages];
+    if (slot == 0) {
+      cfg.gridDim = dim3(2 * (dev.sms / 2));
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(prefix pair)");
+      slot = n > 0 ? n : -1;
+    }
+    resident = slot;
+  }
+  if (resident <= 0) return PA_ERR_UNSUPPORTED;
+
+  CUtensorMap tm_k, tm_v;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.BS;
+  const int box_rows = a.BS < pa::kChunkTokens ? a.BS : pa::kChunkTokens;
+  pa_status st = make_cache_map<T>(&tm_k, a.k_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  st = make_cache_map<T>(&tm_v, a.v_cache, D, a.Hkv, rows, 1, true, box_rows);
+  if (st != PA_OK) return st;
+  CUtensorMap tm_q;
+  st = make_query_map<T>(&tm_q, a.q, a.S, a.Hq, D, G);
+  if (st != PA_OK) return st;
+  const int np = a.total_parts;
+  const size_t acc_elems = static_cast<size_t>(a.S) * a.Hq * np * D;
+  char* ws = static_cast<char*>(a.workspace);
+  const size_t list_bytes = units_bytes(a.S, a.Hq, max_parts(a.max_blocks, a.BS, a.P));
+  pa::PrefixParams prm;
+  prm.q = a.q;
+  prm.prefix_blocks = pf.prefix_blocks;
+  prm.part_acc = reinterpret_cast<float*>(ws + kSchedBytes + list_bytes);
+  prm.part_ml = reinterpret_cast<float2*>(prm.part_acc + acc_elems);
+  prm.num_seqs = a.S;
+  prm.num_q_heads = a.Hq;
+  prm.num_kv_heads = a.Hkv;
+  prm.block_size = a.BS;
+  prm.num_blocks = a.num_blocks;
+  prm.prefix_len = pf.prefix_len;
+  prm.split_tokens = kPrefixSplitTokens;
+  prm.max_parts = np;
+  prm.stages = stages;
+  prm.stage_bytes = static_cast<uint32_t>(pa::kUmmaTile * D * sizeof(T) / 2);
+  prm.qk_scale = a.scale * 1.4426950408889634f;
+  prm.row_pairs = (a.S * G + pa::kPairRows - 1) / pa::kPairRows;
+  prm.num_splits = prefix_splits(pf.prefix_len);
+  prm.num_units = static_cast<long long>(prm.row_pairs) * a.Hkv * prm.num_splits;
+  // a multiple of the pairs per head, so that the clusters that read the same
+  // (head, slice) for different pairs are at the same offset of their shares
+  int clusters = resident;
+  if (prm.row_pairs <= clusters) clusters = clusters / prm.row_pairs * prm.row_pairs;
+  if (prm.num_units < clusters) clusters = static_cast<int>(prm.num_units);
+  cfg.gridDim = dim3(2 * clusters);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_k, tm_v, tm_q, prm);
+  if (e != cudaSuccess) return cuda_fail(e, "prefix_pair_kernel launch");
+  g_last_prefix_kernel = 1;
   return PA_OK;
 }
 
@@ -120,7 +220,14 @@ pa_status launch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   DeviceInfo dev;
   pa_status st = device_info(&dev);
   if (st != PA_OK) return st;
-  if (prefix_uses_umma()) return launch_prefix_umma<T, D, G>(a, pf, dev);
+  const PrefixPath path = prefix_path();
+  if constexpr (D == 128) {
+    if (path == PrefixPath::kPair) {
+      st = launch_prefix_pair<T, G>(a, pf, dev);
+      if (st != PA_ERR_UNSUPPORTED) return st;
+    }
+  }
+  if (path != PrefixPath::kMma) return launch_prefix_umma<T, D, G>(a, pf, dev);
   const size_t stage_bytes = static_cast<size_t>(pa::kPrefixTile) * D * sizeof(T);
   int stages = 3;
   const int forced_st = env_int("PA_PREFIX_STAGES");
@@ -164,6 +271,7 @@ pa_status launch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   kern<<<grid, (pa::kPrefixWarps + 1) * 32, smem, a.stream>>>(tm_k, tm_v, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefix_attention_kernel launch");
+  g_last_prefix_kernel = 3;
   return PA_OK;
 }
 
@@ -435,6 +543,8 @@ pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, 
   st = dtype == PA_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
   return st == PA_OK ? pa::ok() : st;
 }
+
+int pa_debug_last_prefix_kernel(void) { return g_last_prefix_kernel; }
 
 pa_status pa_debug_decode_stall(int64_t wait_limit_ns) {
   if (wait_limit_ns != 0 && (wait_limit_ns < 1000 || wait_limit_ns > static_cast<int64_t>(pa::kWaitLimitNs)))

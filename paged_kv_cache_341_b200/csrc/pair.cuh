@@ -1,0 +1,133 @@
+// Two-CTA (SM pair) building blocks for sm_100a: cluster rank and barrier,
+// mbarrier arrivals on the peer CTA's shared memory, and the cta_group::2
+// forms of the tensor-memory allocation, the MMA and its commit, in which one
+// thread of the even CTA drives the tensor cores of both SMs of a cluster of
+// two (M = 256: each SM computes its own 128 rows; the B operand is split
+// between the two CTAs' shared memory by N).
+#ifndef PAGEDATTN_PAIR_CUH
+#define PAGEDATTN_PAIR_CUH
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace pa {
+namespace pair {
+
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The shared::cluster address of the variable at `p` (this CTA's shared
+// memory) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (this CTA's or
+// the peer's), with the instruction's default (release) semantics.  What the
+// arrival announces is never a generic-proxy write: it is tensor-memory
+// writes (P, after tcgen05.wait::st and tcgen05.fence::before_thread_sync),
+// tensor-memory reads, or the completion of a TMA copy the arriving thread
+// has observed; a release at cluster scope here was measured to stall the
+// arriving warp for ~1,800 cycles.
+__device__ __forceinline__ void arrive_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity);
+}
+
+// Bounded wait like mbar_wait, for barriers the peer CTA arrives on.
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             uint64_t limit_ns = kWaitLimitNs) {
+  if (try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      set_device_error(DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Every thread of both CTAs; barrier initialisation and earlier shared-memory
+// writes of either CTA are visible to the other afterwards.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+}  // namespace pair
+
+namespace tc {
+
+// Tensor memory of both SMs of the pair, the same columns in each: one full
+// warp with the same warp index in each CTA.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem] over the pair (M = 256): each CTA's A is its
+// 128 rows at the same shared-memory offset, each CTA's B its half of N.
+__device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  const uint32_t z = 0u;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z)
+      : "memory");
+}
+
+// The same with A in tensor memory (each CTA's rows in its own columns).
+__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  const uint32_t z = 0u;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at the same offset in each CTA of `cta_mask`
+// when every pair-mode tcgen05 operation this thread issued has completed.
+__device__ __forceinline__ void commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+}  // namespace tc
+}  // namespace pa
+
+#endif

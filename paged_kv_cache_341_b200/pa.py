@@ -65,6 +65,7 @@ SIGNATURES = {
                                                  _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _i32, _vp]),
     "pa_device_error": (_i32, [_p32, _i32]),
     "pa_debug_decode_stall": (_i32, [_i64]),
+    "pa_debug_last_prefix_kernel": (_i32, []),
     "pa_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in SIGNATURES.items():
@@ -399,6 +400,11 @@ def pa_device_error(reset=True):
     code = ctypes.c_int32()
     _check(_lib.pa_device_error(ctypes.byref(code), 1 if reset else 0))
     return code.value
+
+
+def pa_debug_last_prefix_kernel():
+    """1 = SM-pair tcgen05 prefix kernel, 2 = one-SM tcgen05, 3 = mma.sync, 0 = none yet (this thread)."""
+    return int(_lib.pa_debug_last_prefix_kernel())
 
 
 def pa_debug_decode_stall(wait_limit_ns):

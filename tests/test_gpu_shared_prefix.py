@@ -26,9 +26,10 @@ def pa():
     return mod
 
 
-@pytest.fixture(params=["umma", "mma"])
+@pytest.fixture(params=["umma", "pair", "mma"])
 def prefix_path(request, monkeypatch):
-    """Run a test once on the tcgen05 (tensor-memory) prefix kernel and once on the mma.sync one."""
+    """Run a test on each prefix kernel: the one-SM tcgen05 kernel (the default), the SM-pair tcgen05
+    kernel (head_dim 128; 64 falls back to the one-SM kernel) and the mma.sync one."""
     monkeypatch.setenv("PA_PREFIX_PATH", request.param)
     return request.param
 
@@ -78,6 +79,15 @@ def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed
 
 SUFFIXES = [0, 1, 15, 16, 17, 100, 33]
 
+# pa_debug_last_prefix_kernel per path; the SM-pair kernel takes head_dim 128
+# only (64 falls back to the one-SM kernel), and on a B200 it always launches
+LAUNCHED = {"pair": 1, "umma": 2, "mma": 3}
+
+
+def check_launched(pa, prefix_path, d):
+    want = LAUNCHED[prefix_path] if not (prefix_path == "pair" and d != 128) else LAUNCHED["umma"]
+    assert pa.pa_debug_last_prefix_kernel() == want, (prefix_path, d, pa.pa_debug_last_prefix_kernel())
+
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("d", [64, 128])
@@ -89,6 +99,7 @@ def test_shared_prefix_matches_oracle(pa, prefix_path, dtype, d, hq, hkv, bs, pr
     # 1056 = 1024 + 32: the second slice ends in a 32-token tile; 1088 ends on a full one
     gpu, ref, plain = run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, SUFFIXES, partition,
                                   seed=prefix_len + bs + hq + d + partition)
+    check_launched(pa, prefix_path, d)
     tag = "%s dtype=%s d=%d hq=%d hkv=%d bs=%d prefix=%d p=%d" % (prefix_path, dtype, d, hq, hkv, bs, prefix_len,
                                                                   partition)
     assert_close(gpu, ref, dtype, tag)
@@ -102,6 +113,7 @@ def test_many_sequences_and_row_tiles(pa, prefix_path, nseq):
     rng = np.random.default_rng(5)
     suffixes = [int(x) for x in rng.integers(0, 600, size=nseq)]
     gpu, ref, _ = run_cascade(pa, "bf16", 32, 8, 128, 16, 2048 + 64, suffixes, 512, seed=6 + nseq)
+    check_launched(pa, prefix_path, 128)
     assert_close(gpu, ref, "bf16", "%d sequences" % nseq)
 
 
@@ -109,6 +121,7 @@ def test_large_scores_rescale_in_tensor_memory(pa, prefix_path):
     # queries scaled up so the running maximum moves by more than 2^8 between
     # tiles: the tcgen05 kernel rescales O inside tensor memory
     gpu, ref, _ = run_cascade(pa, "bf16", 16, 4, 128, 16, 1024 + 512, [3, 0, 40], 0, seed=8, q_scale=12.0)
+    check_launched(pa, prefix_path, 128)
     assert_close(gpu, ref, "bf16", "large scores")
 
 
