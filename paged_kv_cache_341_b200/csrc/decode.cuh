@@ -1172,13 +1172,89 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams prm
   }
 }
 
+// The planner for batches of at most 32 sequences: the same list as
+// plan_kernel (full partitions in sequence order, then one remainder entry
+// per sequence, larger remainders first) worked out by one warp with
+// shuffles, so the decode grid waits for one warp's loads and stores rather
+// than a 1,024-thread block's scans.  Same speculative protocol: the plan is
+// worked out from lengths read before griddepcontrol.wait, the lengths are
+// read again after it, and the plan is redone if any changed; nothing is
+// written before the wait.
+constexpr int kPlanSmallSeqs = 32;
+
+__global__ void __launch_bounds__(32) plan_small_kernel(const PlanParams prm) {
+  allow_dependent_launch();                    // the decode grid may launch; it waits for this one
+  const int lane = threadIdx.x;
+  const int S = prm.num_seqs, P = prm.partition_size, nt = prm.num_tiles;
+  const bool mine = lane < S;
+  auto load_len = [&]() {
+    int len = mine ? __ldcg(prm.context_lens + lane) : 0;
+    return len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
+  };
+  const int full_chunks = P / kChunkTokens;
+  int len = 0, nfull = 0, base = 0, written = 0, pos = -1, tot = 0, work = 0, umax = 1;
+  bool waited = false;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    len = load_len();
+    nfull = P > 0 ? len / P : 0;
+    // remainder bucket (16-token chunks, largest last bucket shared), -1 if none
+    int key = -1, rc = 0;
+    if (mine && !(P > 0 && len > 0 && len % P == 0)) {
+      const int rem = P > 0 ? len % P : len;
+      const int chunks = (rem + kChunkTokens - 1) / kChunkTokens;
+      key = chunks < kPlanBuckets ? chunks : kPlanBuckets - 1;
+      rc = chunks > 1 ? chunks : 1;
+    }
+    // full entries: exclusive scan of nfull over the lanes
+    int incl = nfull;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    base = incl - nfull;
+    written = __shfl_sync(0xffffffffu, incl, 31);
+    // remainder position: after every entry with a larger bucket, or the same bucket and a lower lane
+    int rank = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int kj = __shfl_sync(0xffffffffu, key, j);
+      rank += (kj >= 0 && (kj > key || (kj == key && j < lane))) ? 1 : 0;
+    }
+    tot = __popc(__ballot_sync(0xffffffffu, key >= 0));
+    pos = key >= 0 ? written + rank : -1;
+    int w = nfull * full_chunks + rc;
+    int um = max(nfull > 0 ? full_chunks : 0, rc);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      w += __shfl_xor_sync(0xffffffffu, w, off);
+      um = max(um, __shfl_xor_sync(0xffffffffu, um, off));
+    }
+    work = w;
+    umax = um > 0 ? um : 1;
+    if (waited) break;
+    wait_prerequisite_grids();                 // the kernel before has finished and its writes are visible
+    waited = true;
+    if (!__any_sync(0xffffffffu, load_len() != len)) break;
+  }
+  if (lane == 0) {
+    prm.header[0] = 0;
+    prm.header[1] = (written + tot) * nt;
+    prm.header[2] = plan_working_grid(prm, tot, work, umax);
+  }
+  if (mine) {
+    for (int p = 0; p < nfull; ++p) prm.units[base + p] = make_int4(lane, p, 0, len);
+    if (pos >= 0) prm.units[pos] = make_int4(lane, nfull, 0, len);
+  }
+}
+
 // ===========================================================================
 // Merge of per-partition partials: M = max m_p, w_p = 2^(m_p - M),
 // out = sum_p w_p acc_p / sum_p w_p l_p.  A CTA of 8 warps covers 8 / W query
 // heads of one sequence with W warps per head (W from the partition count the
 // workspace allows: 1 up to 8 partitions, up to 8 for 33 or more); the W warps
-// of a head each take every W-th partition with four rows in flight, and sum
-// their parts through shared memory.  Sequences that fit one partition were
+// of a head each take every W-th partition, eight rows at a time loaded
+// together with the (m, l) pairs (one round of loads up to 8 W partitions),
+// and sum their parts through shared memory.  Sequences that fit one partition were
 // written by the decode kernel and are skipped.  Launched as a programmatic
 // dependent of the decode kernel: it reads nothing before griddepcontrol.wait
 // has returned, i.e. before that grid (and so everything before it on the
@@ -1223,66 +1299,62 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
   float mx = -INFINITY, lsum = 0.f;
   if (active) {
-    // every warp of the head computes M and L over all partitions in one
-    // sweep of the (m, l) pairs: each lane keeps a running maximum and a sum
-    // rescaled to it, and the lanes' pairs are merged the same way
-    for (int p = lane; p < np; p += 32) {
-      const float2 ml = prm.part_ml[base + p];
-      if (ml.x > mx) {
-        lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
-        mx = ml.x;
-      } else if (ml.x != -INFINITY) {
-        lsum += ml.y * exp2_approx(ml.x - mx);
-      }
-    }
+    // This warp's partitions are sub, sub + wph, ...; their rows are loaded
+    // kMergeRows at a time, together with the (m, l) pairs that every warp of
+    // the head sweeps for M and L (each lane keeps a running maximum and a sum
+    // rescaled to it, and the lanes' pairs are merged the same way), so that a
+    // head with up to kMergeRows * wph partitions is merged after one round
+    // of loads.  A partition with m = -inf holds no token (a slot the
+    // shared-prefix kernel left empty, or never written): its row is read but
+    // never used.
+    constexpr int kMergeRows = 8;
+    const int K = np > sub ? (np - sub + wph - 1) / wph : 0;
+    for (int k0 = 0; k0 < K; k0 += kMergeRows) {
+      float2 v[kMergeRows][PER / 2];
+      float mk[kMergeRows];
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
-      const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
-      const float mn = fmaxf(mx, mo);
-      lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) + (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
-      mx = mn;
-    }
-    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
-    // this warp's partitions sub, sub + wph, ... that hold tokens, four rows
-    // in flight.  A partition with m = -inf holds none (a slot the
-    // shared-prefix kernel left empty): it is found from a ballot over the
-    // (m, l) pairs and its row is never read.
-    const unsigned share = wph == 1 ? 0xffffffffu
-                                    : (wph == 2 ? 0x55555555u : (wph == 4 ? 0x11111111u : 0x01010101u)) << sub;
-    for (int p0 = 0; p0 < np; p0 += 32) {
-      const int pl = p0 + lane;
-      const float ml_x = pl < np ? prm.part_ml[base + pl].x : -INFINITY;
-      unsigned todo = __ballot_sync(0xffffffffu, ml_x != -INFINITY) & share;
-      while (todo) {
-        int pk[4];
-        int n = 0;
+      for (int u = 0; u < kMergeRows; ++u) {
+        const int pp = sub + wph * (k0 + u);
+        mk[u] = -INFINITY;
+        if (k0 + u < K) {
+          const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pp) * D + lane * PER);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          pk[u] = todo ? __ffs(todo) - 1 : -1;
-          if (todo) {
-            todo &= todo - 1;
-            ++n;
-          }
-        }
-        float2 v[4][PER / 2];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (u < n) {
-            const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + pk[u]) * D + lane * PER);
-#pragma unroll
-            for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (u < n) {
-            const float wu = exp2_approx(__shfl_sync(0xffffffffu, ml_x, pk[u]) - mx);
-#pragma unroll
-            for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
-          }
+          for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+          mk[u] = prm.part_ml[base + pp].x;
         }
       }
+      if (k0 == 0) {
+        for (int p = lane; p < np; p += 32) {
+          const float2 ml = prm.part_ml[base + p];
+          if (ml.x > mx) {
+            lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
+            mx = ml.x;
+          } else if (ml.x != -INFINITY) {
+            lsum += ml.y * exp2_approx(ml.x - mx);
+          }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+          const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
+          const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
+          const float mn = fmaxf(mx, mo);
+          lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) +
+                 (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
+          mx = mn;
+        }
+        if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeRows; ++u) {
+        if (mk[u] != -INFINITY) {
+          const float wu = exp2_approx(mk[u] - mx);
+#pragma unroll
+          for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
+        }
+      }
+    }
+    if (K == 0) {
+      // a warp without partitions still needs M and L for nothing; no output from it
     }
   }
   if (wph > 1) {

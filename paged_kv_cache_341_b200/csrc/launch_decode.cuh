@@ -277,11 +277,16 @@ pa_status launch_decode(const DecodeArgs& a) {
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t pcfg = {};
     pcfg.gridDim = dim3(1);
-    pcfg.blockDim = dim3(pa::kPlanThreads);
     pcfg.stream = a.stream;
     pcfg.attrs = pdl;
     pcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&pcfg, pa::plan_kernel, pp);
+    if (a.S <= pa::kPlanSmallSeqs) {
+      pcfg.blockDim = dim3(32);
+      e = cudaLaunchKernelEx(&pcfg, pa::plan_small_kernel, pp);
+    } else {
+      pcfg.blockDim = dim3(pa::kPlanThreads);
+      e = cudaLaunchKernelEx(&pcfg, pa::plan_kernel, pp);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
