@@ -1253,8 +1253,9 @@ __global__ void __launch_bounds__(32) plan_small_kernel(const PlanParams prm) {
 // heads of one sequence with W warps per head (W from the partition count the
 // workspace allows: 1 up to 8 partitions, up to 8 for 33 or more); the W warps
 // of a head each take every W-th partition, eight rows at a time loaded
-// together with the (m, l) pairs (one round of loads up to 8 W partitions),
-// and sum their parts through shared memory.  Sequences that fit one partition were
+// together with the (m, l) pairs (one round of loads up to 8 W partitions;
+// with shared-prefix slots the pairs first, and only the non-empty rows), and
+// sum their parts through shared memory.  Sequences that fit one partition were
 // written by the decode kernel and are skipped.  Launched as a programmatic
 // dependent of the decode kernel: it reads nothing before griddepcontrol.wait
 // has returned, i.e. before that grid (and so everything before it on the
@@ -1283,78 +1284,157 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
   __shared__ float2 s_sum[kReduceWarps][D / 2];
   const int s = blockIdx.y;
-  wait_prerequisite_grids();                 // the decode grid (and all before it) is done and visible
-  int len = prm.context_lens[s];
-  len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
-  const int np = prm.part_offset + parts_of(len, prm.partition_size);
-  if (prm.part_offset == 0 && np <= 1) return;          // the same for the whole CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wph = prm.warps_per_head;
   const int hq = blockIdx.x * (kReduceWarps / wph) + warp / wph;
   const int sub = warp & (wph - 1);
   const bool active = hq < prm.num_q_heads;
   const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + (active ? hq : 0)) * prm.max_parts;
+  const bool dense = prm.part_offset == 0;   // every slot below np holds a partition
+  wait_prerequisite_grids();                 // the decode grid (and all before it) is done and visible
+  // Dense calls: the first round of this warp's rows (sub, sub + wph, ...),
+  // their m and the first 64 (m, l) pairs are loaded together with the
+  // length, within the head's max_parts slots; what lies at or past the
+  // sequence's partition count is not used.
+  constexpr int kMergeRows = 8;
+  float2 v[kMergeRows][PER / 2];
+  float mk[kMergeRows];
+  float2 sw0 = make_float2(-INFINITY, 0.f), sw1 = make_float2(-INFINITY, 0.f);
+  if (dense && active) {
+#pragma unroll
+    for (int u = 0; u < kMergeRows; ++u) {
+      const int pp = sub + wph * u;
+      mk[u] = -INFINITY;
+      if (pp < prm.max_parts) {
+        const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pp) * D + lane * PER);
+#pragma unroll
+        for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+        mk[u] = prm.part_ml[base + pp].x;
+      }
+    }
+    if (lane < prm.max_parts) sw0 = prm.part_ml[base + lane];
+    if (lane + 32 < prm.max_parts) sw1 = prm.part_ml[base + lane + 32];
+  }
+  int len = prm.context_lens[s];
+  len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
+  const int np = prm.part_offset + parts_of(len, prm.partition_size);
+  if (dense && np <= 1) return;              // the same for the whole CTA
   float2 o[PER / 2];
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
   float mx = -INFINITY, lsum = 0.f;
-  if (active) {
-    // This warp's partitions are sub, sub + wph, ...; their rows are loaded
-    // kMergeRows at a time, together with the (m, l) pairs that every warp of
-    // the head sweeps for M and L (each lane keeps a running maximum and a sum
-    // rescaled to it, and the lanes' pairs are merged the same way), so that a
-    // head with up to kMergeRows * wph partitions is merged after one round
-    // of loads.  A partition with m = -inf holds no token (a slot the
-    // shared-prefix kernel left empty, or never written): its row is read but
-    // never used.
-    constexpr int kMergeRows = 8;
+  if (active && dense) {
+    // M and L in one sweep of the (m, l) pairs (each lane keeps a running
+    // maximum and a sum rescaled to it, and the lanes' pairs are merged the
+    // same way); then this warp's rows, kMergeRows at a time (one round of
+    // loads for a head with up to kMergeRows * wph partitions)
+    auto take = [&](float2 ml) {
+      if (ml.x > mx) {
+        lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
+        mx = ml.x;
+      } else if (ml.x != -INFINITY) {
+        lsum += ml.y * exp2_approx(ml.x - mx);
+      }
+    };
+    if (lane < np) take(sw0);
+    if (lane + 32 < np) take(sw1);
+    for (int p = lane + 64; p < np; p += 32) take(prm.part_ml[base + p]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
+      const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
+      const float mn = fmaxf(mx, mo);
+      lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) +
+             (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
+      mx = mn;
+    }
+    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
     const int K = np > sub ? (np - sub + wph - 1) / wph : 0;
     for (int k0 = 0; k0 < K; k0 += kMergeRows) {
-      float2 v[kMergeRows][PER / 2];
-      float mk[kMergeRows];
+      if (k0 > 0) {
 #pragma unroll
-      for (int u = 0; u < kMergeRows; ++u) {
-        const int pp = sub + wph * (k0 + u);
-        mk[u] = -INFINITY;
-        if (k0 + u < K) {
-          const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pp) * D + lane * PER);
+        for (int u = 0; u < kMergeRows; ++u) {
+          const int pp = sub + wph * (k0 + u);
+          mk[u] = -INFINITY;
+          if (k0 + u < K) {
+            const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pp) * D + lane * PER);
 #pragma unroll
-          for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
-          mk[u] = prm.part_ml[base + pp].x;
-        }
-      }
-      if (k0 == 0) {
-        for (int p = lane; p < np; p += 32) {
-          const float2 ml = prm.part_ml[base + p];
-          if (ml.x > mx) {
-            lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
-            mx = ml.x;
-          } else if (ml.x != -INFINITY) {
-            lsum += ml.y * exp2_approx(ml.x - mx);
+            for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+            mk[u] = prm.part_ml[base + pp].x;
           }
         }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
-          const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
-          const float mn = fmaxf(mx, mo);
-          lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) +
-                 (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
-          mx = mn;
-        }
-        if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
       }
 #pragma unroll
       for (int u = 0; u < kMergeRows; ++u) {
-        if (mk[u] != -INFINITY) {
+        if (k0 + u < K && mk[u] != -INFINITY) {
           const float wu = exp2_approx(mk[u] - mx);
 #pragma unroll
           for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
         }
       }
     }
-    if (K == 0) {
-      // a warp without partitions still needs M and L for nothing; no output from it
+  } else if (active) {
+    // Shared-prefix slots, most of them empty (m = -inf, left so by the
+    // prefix kernel's segments): the (m, l) sweep first, then only the rows
+    // of slots that hold tokens, found by a ballot.  Every warp of the head
+    // computes M and L in one sweep as above.
+    for (int p = lane; p < np; p += 32) {
+      const float2 ml = prm.part_ml[base + p];
+      if (ml.x > mx) {
+        lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
+        mx = ml.x;
+      } else if (ml.x != -INFINITY) {
+        lsum += ml.y * exp2_approx(ml.x - mx);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
+      const float lo = __shfl_xor_sync(0xffffffffu, lsum, off);
+      const float mn = fmaxf(mx, mo);
+      lsum = (mx == -INFINITY ? 0.f : lsum * exp2_approx(mx - mn)) + (mo == -INFINITY ? 0.f : lo * exp2_approx(mo - mn));
+      mx = mn;
+    }
+    if (mx == -INFINITY) mx = 0.f;          // no partition saw a token: all weights are 0
+    // this warp's partitions sub, sub + wph, ... that hold tokens, four rows
+    // in flight.  A partition with m = -inf holds none (a slot the
+    // shared-prefix kernel left empty): it is found from a ballot over the
+    // (m, l) pairs and its row is never read.
+    const unsigned share = wph == 1 ? 0xffffffffu
+                                    : (wph == 2 ? 0x55555555u : (wph == 4 ? 0x11111111u : 0x01010101u)) << sub;
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      const int pl = p0 + lane;
+      const float ml_x = pl < np ? prm.part_ml[base + pl].x : -INFINITY;
+      unsigned todo = __ballot_sync(0xffffffffu, ml_x != -INFINITY) & share;
+      while (todo) {
+        int pk[4];
+        int n = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          pk[u] = todo ? __ffs(todo) - 1 : -1;
+          if (todo) {
+            todo &= todo - 1;
+            ++n;
+          }
+        }
+        float2 v[4][PER / 2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (u < n) {
+            const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + p0 + pk[u]) * D + lane * PER);
+#pragma unroll
+            for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (u < n) {
+            const float wu = exp2_approx(__shfl_sync(0xffffffffu, ml_x, pk[u]) - mx);
+#pragma unroll
+            for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
+          }
+        }
+      }
     }
   }
   if (wph > 1) {
