@@ -1252,8 +1252,8 @@ __global__ void __launch_bounds__(32) plan_small_kernel(const PlanParams prm) {
 // out = sum_p w_p acc_p / sum_p w_p l_p.  A CTA of 8 warps covers 8 / W query
 // heads of one sequence with W warps per head (W from the partition count the
 // workspace allows: 1 up to 8 partitions, up to 8 for 33 or more); the W warps
-// of a head each take every W-th partition, eight rows at a time loaded
-// together with the (m, l) pairs (one round of loads up to 8 W partitions;
+// of a head each take every W-th partition, 4 or 6 rows at a time loaded
+// together with the (m, l) pairs (one round of loads up to 6 W partitions;
 // with shared-prefix slots the pairs first, and only the non-empty rows), and
 // sum their parts through shared memory.  Sequences that fit one partition were
 // written by the decode kernel and are skipped.  Launched as a programmatic
@@ -1278,7 +1278,7 @@ __host__ __device__ constexpr int reduce_warps_per_head(int max_parts) {
   return max_parts <= 8 ? 1 : (max_parts <= 16 ? 2 : (max_parts <= 32 ? 4 : 8));
 }
 
-template <typename T, int D>
+template <typename T, int D, int ROWS>
 __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceParams prm) {
   constexpr int PER = D / 32;                // contiguous elements per lane
   static_assert(PER % 2 == 0, "head_dim must be a multiple of 64");
@@ -1291,34 +1291,40 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
   const bool active = hq < prm.num_q_heads;
   const size_t base = (static_cast<size_t>(s) * prm.num_q_heads + (active ? hq : 0)) * prm.max_parts;
   const bool dense = prm.part_offset == 0;   // every slot below np holds a partition
+  auto clamp_len = [&](int v) { return v < 0 ? 0 : (v > prm.cap ? prm.cap : v); };
+  // the length as it stands (through L2) before the wait: only a guess, as
+  // the kernel before the planner may still be writing it; checked below
+  const int len_guess = dense ? clamp_len(__ldcg(prm.context_lens + s)) : 0;
   wait_prerequisite_grids();                 // the decode grid (and all before it) is done and visible
-  // Dense calls: the first round of this warp's rows (sub, sub + wph, ...),
-  // their m and the first 64 (m, l) pairs are loaded together with the
-  // length, within the head's max_parts slots; what lies at or past the
-  // sequence's partition count is not used.
-  constexpr int kMergeRows = 8;
+  // Dense calls: the first round of this warp's rows (sub, sub + wph, ...)
+  // below the guessed partition count, their m and the first 64 (m, l) pairs
+  // are loaded together with the length; if the length read after the wait
+  // differs, the round is loaded again.
+  constexpr int kMergeRows = ROWS;          // 6 for long contexts, 4 otherwise (registers: CTAs per SM)
   float2 v[kMergeRows][PER / 2];
   float mk[kMergeRows];
   float2 sw0 = make_float2(-INFINITY, 0.f), sw1 = make_float2(-INFINITY, 0.f);
-  if (dense && active) {
+  const int np_guess = parts_of(len_guess, prm.partition_size);
+  auto load_round = [&](int npg) {
 #pragma unroll
     for (int u = 0; u < kMergeRows; ++u) {
       const int pp = sub + wph * u;
       mk[u] = -INFINITY;
-      if (pp < prm.max_parts) {
+      if (pp < npg) {
         const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pp) * D + lane * PER);
 #pragma unroll
         for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
         mk[u] = prm.part_ml[base + pp].x;
       }
     }
-    if (lane < prm.max_parts) sw0 = prm.part_ml[base + lane];
-    if (lane + 32 < prm.max_parts) sw1 = prm.part_ml[base + lane + 32];
-  }
-  int len = prm.context_lens[s];
-  len = len < 0 ? 0 : (len > prm.cap ? prm.cap : len);
+    sw0 = lane < npg ? prm.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
+    sw1 = lane + 32 < npg ? prm.part_ml[base + lane + 32] : make_float2(-INFINITY, 0.f);
+  };
+  if (dense && active && np_guess > 1) load_round(np_guess);
+  const int len = clamp_len(prm.context_lens[s]);
   const int np = prm.part_offset + parts_of(len, prm.partition_size);
   if (dense && np <= 1) return;              // the same for the whole CTA
+  if (dense && active && np != np_guess) load_round(np);
   float2 o[PER / 2];
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) o[e] = make_float2(0.f, 0.f);
@@ -1336,8 +1342,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
         lsum += ml.y * exp2_approx(ml.x - mx);
       }
     };
-    if (lane < np) take(sw0);
-    if (lane + 32 < np) take(sw1);
+    take(sw0);                               // -inf past np
+    take(sw1);
     for (int p = lane + 64; p < np; p += 32) take(prm.part_ml[base + p]);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {

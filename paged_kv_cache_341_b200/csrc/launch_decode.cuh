@@ -333,7 +333,14 @@ pa_status launch_decode(const DecodeArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, D>, rp);
+    // six rows a warp in flight where a head has more than 16 partitions (one
+    // round of loads for up to 48 partitions; 64 registers, so a 70B-shaped
+    // merge of 512 CTAs is one wave), four otherwise (48 registers)
+    if (rp.warps_per_head >= 4) {
+      e = cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, D, 6>, rp);
+    } else {
+      e = cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, D, 4>, rp);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "reduce_kernel launch");
   }
 
