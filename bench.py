@@ -294,15 +294,33 @@ class ReferenceScenario:
         self.cache = type("HostTables", (), {"tables": tables, "lens": lens})()
         used = sorted({int(b) for r in range(rows) for b in tables[r, :-(-int(lens[r]) // w.block_size)]})
         self.k_host, self.v_host = workloads.fill_blocks(w, used, w.seed + 100)
+        # the step the GPU arm times: one slot reserved per sequence (copy-on-write of a shared partly
+        # filled block), the step's new K/V written there, attention over len + 1 tokens
+        _, k_new, v_new = self.step_inputs(0)
+        kf = self.k_host.view(-1, w.num_kv_heads, w.head_dim)
+        vf = self.v_host.view(-1, w.num_kv_heads, w.head_dim)
+        for i, r in enumerate(range(self.rows.start, self.rows.stop)):
+            n = int(lens[r])
+            table = [int(x) for x in tables[r, :-(-n // w.block_size)]]
+            slot, n1, src, dst = op.reserve_slot(table, n, w.max_blocks_per_seq)
+            if src >= 0:
+                self.k_host[dst] = self.k_host[src]
+                self.v_host[dst] = self.v_host[src]
+            kf[slot] = k_new[i]
+            vf[slot] = v_new[i]
+            tables[r, :len(table)] = table
+            lens[r] = n1
 
     @property
     def batch(self):
         return self.rows.stop - self.rows.start
 
     def step_inputs(self, step):
+        """The GPU scenario's seeded inputs of step ``step``: q, k_new, v_new."""
         from paged_kv_cache_341_b200 import workloads
         seed = self.w.seed + 1000 + 10 * step
-        return workloads.queries(self.w, seed, num_seqs=self.batch), None, None
+        k_new, v_new = workloads.new_tokens(self.w, seed + 3, self.batch)
+        return workloads.queries(self.w, seed, num_seqs=self.batch), k_new, v_new
 
 
 def workload_config(sc, args, l2_bytes=None):
