@@ -20,7 +20,7 @@
 // on S(t)), and the softmax runs four threads per row.
 //
 // Measured on the 200-sequence, 30,720-token shared-prefix step (B200): a
-// cascade call of 0.246 ms against 0.241 ms with the one-SM kernel.  The
+// cascade call of 0.231 ms against 0.225 ms with the one-SM kernel.  The
 // halved K/V loads do not pay because the softmax bounds both: here a
 // 128-row x 128-token tile takes ~2.4K cycles of softmax (its exponentials
 // alone ~900 cycles per SM sub-partition at one MUFU instruction per 8
