@@ -39,28 +39,6 @@ __device__ __forceinline__ void arrive_cluster(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity);
-}
-
-// Bounded wait like mbar_wait, for barriers the peer CTA arrives on.
-__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                             uint64_t limit_ns = kWaitLimitNs) {
-  if (try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (try_wait_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      *abort_flag = 1;
-      set_device_error(DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // Every thread of both CTAs; barrier initialisation and earlier shared-memory
 // writes of either CTA are visible to the other afterwards.
 __device__ __forceinline__ void cluster_sync() {

@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       uint32_t kph = 0, vph = 0;
       int tau_s = 0, tau_p = 0;
       auto issue_s = [&](int qb) {
-        if (!pair::wait_cluster(&k_full[kst], kph, abort_flag)) return false;
+        if (!mbar_wait(&k_full[kst], kph, abort_flag)) return false;
         tc::fence_after_sync();
         const uint64_t kb = k_desc + ((kst * kKHalf) >> 4);
         const uint64_t qbd = q_desc + ((qb * kQBytes) >> 4);
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const PrefixSegment I = prefix_pair_segment<G>(u, u_end, prm);
         u = I.end;
         const int qb = items & 1;
-        if (!pair::wait_cluster(&q_full[qb], (items >> 1) & 1, abort_flag)) {
+        if (!mbar_wait(&q_full[qb], (items >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -396,9 +396,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (!ok) break;
         if (n <= 2) tc::commit_pair(&q_empty[qb], kBoth);
         for (int j = 0; j < n; ++j) {
-          if (!pair::wait_cluster(&v_full[vst], vph, abort_flag) ||
-              !pair::wait_cluster(&p_full[tau_p & 1], (tau_p >> 1) & 1, abort_flag) ||
-              (j == 0 && items > 0 && !pair::wait_cluster(o_free, (items - 1) & 1, abort_flag))) {
+          if (!mbar_wait(&v_full[vst], vph, abort_flag) ||
+              !mbar_wait(&p_full[tau_p & 1], (tau_p >> 1) & 1, abort_flag) ||
+              (j == 0 && items > 0 && !mbar_wait(o_free, (items - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
