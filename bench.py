@@ -69,19 +69,21 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def call_label(cascade, w, calls, peak_kind):
+def call_label(cascade, w, batch, calls, peak_kind):
     """What the roofline's achieved figure times."""
     decode = ("decode_mma_kernel" if w.elem_bytes == 2 and os.environ.get("PA_DECODE_PATH") != "alu"
               else "decode_kernel")
+    # the one-warp planner serves batches of up to 32 sequences
+    planner = "plan_small_kernel" if batch <= 32 else "plan_kernel"
     if cascade:
         prefix = {"mma": "prefix_attention_kernel", "pair": "prefix_pair_kernel"}.get(
             os.environ.get("PA_PREFIX_PATH", ""), "prefix_umma_kernel")
-        return ("pa_decode_attention_shared_prefix call (%s + plan_kernel + %s + reduce_kernel), median of %d "
+        return ("pa_decode_attention_shared_prefix call (%s + %s + %s + reduce_kernel), median of %d "
                 "calls; achieved counts the logical K/V bytes of every sequence (the shared prefix once per "
                 "sequence), so a frac above 1 measures the sharing, not HBM; peak = %s copy bandwidth"
-                % (prefix, decode, calls, peak_kind))
-    return ("pa_decode_attention call (plan_kernel + %s + reduce_kernel), median of %d calls; peak = %s copy "
-            "bandwidth" % (decode, calls, peak_kind))
+                % (prefix, planner, decode, calls, peak_kind))
+    return ("pa_decode_attention call (%s + %s + reduce_kernel), median of %d calls; peak = %s copy "
+            "bandwidth" % (planner, decode, calls, peak_kind))
 
 
 def traffic_record(workload):
@@ -532,7 +534,7 @@ def run_ours(args):
             "decode_tokens_per_s": round(world * sc.batch / (ms / 1e3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": call_label(cascade, w, len(att_times), peak_kind),
+                         "kernel": call_label(cascade, w, sc.batch, len(att_times), peak_kind),
                          "timed_calls": len(att_times),
                          "statistic": "median",
                          "call_ms": {"median": round(float(np.median(att_times)), 5),
