@@ -15,17 +15,40 @@
 //                    by N: CTA r holds head dimensions 64 r .. 64 r + 63
 // so each SM loads half of every K/V tile (16 KB of K, 16 KB of V) where the
 // one-SM form loads all of it for 128 rows, and each SM's tensor core still
-// works on a full M 128 x N 128 tile.  Each CTA has one query tile and two
-// score buffers in tensor memory (S(t+1) is computed while the softmax works
-// on S(t)), and the softmax runs four threads per row.
+// works on a full M 128 x N 128 tile.
+//
+// Tensor memory (per SM): score buffers S_0, S_1 (columns 0..255) and
+// accumulators O_0, O_1 (256..511).  Token tile t, counted over the CTA's
+// whole share, goes to S_{t mod 2} and PV(t) accumulates into O_{t mod 2}.
+// The softmax is two groups of eight warps: group g takes the tiles with
+// t mod 2 = g with its own reference maximum and sum, so that one group's
+// exponentials overlap the other group's tensor-memory loads, maximum
+// exchange and stores.  In a group two threads share a query row (a
+// tensor-memory lane): half h takes scores 64 h .. 64 h + 63, 32 at a time,
+// and the two exchange their maxima through shared memory.  The reference
+// maximum moves only when a scaled score passes it by 2^8 (the decode
+// kernel's rule); then the thread rescales its half of O_g once the group's
+// previous PV has completed.  Weights rounded to the cache's 16-bit type go
+// over the thread's own scores (tokens 64 h + 32 c + 2j, + 2j + 1 in column
+// 64 h + 32 c + j) as the A operand of PV; the row sums take the weights
+// before rounding.  At the end of a segment all four threads of a row
+// exchange (m, l) and each writes a quarter of the partial,
+// 2^(m_0 - M) O_0 + 2^(m_1 - M) O_1 with M = max(m_0, m_1).
 //
 // Measured on the 200-sequence, 30,720-token shared-prefix step (B200): a
-// cascade call of 0.231 ms against 0.225 ms with the one-SM kernel.  The
-// halved K/V loads do not pay because the softmax bounds both: here a
-// 128-row x 128-token tile takes ~2.4K cycles of softmax (its exponentials
-// alone ~900 cycles per SM sub-partition at one MUFU instruction per 8
-// cycles, with the four warps of a sub-partition in the same phase), against
-// ~1.5K cycles of products.  The work split (stream-K shares of (query-tile
+// cascade call of 0.2253 ms against 0.2262 ms with the one-SM kernel on the
+// same box (with one softmax group of sixteen warps over both score buffers:
+// 0.231 against 0.225 ms).  Clock stamps per tile show each group busy
+// ~2.2K of its ~4.5K-cycle period (loads and maximum ~440, exchange ~300,
+// exponentials and stores ~1.3K) and the issuing thread spending ~1.3K cycles
+// per tile in the sixteen M 256 x N 128 x K 16 products (about 80-87 cycles
+// each, whether the pipe was idle or not) and the rest waiting for weights,
+// V and K or committing; a second issuing warp for the S products was
+// measured slower (0.228 against 0.224 ms on its box).  Stamps of %globaltimer
+// and clock64 per CTA put the SM clock over the kernel at ~1.75 GHz (the
+// step draws 965-990 W of the 1 kW limit), the first S product 4.9 us after
+// launch, and the CTAs' last tiles between 138 and 160 us (per-unit times
+// differ by +-7 % between clusters).  The work split (stream-K shares of (query-tile
 // pair, KV head, 512-token slice) units, segments accumulated into one
 // partial each) is that of the one-SM form.
 //
@@ -37,8 +60,9 @@
 // relays the completion of that CTA's own copies (which arrive on its own
 // barriers, so that it can wait for them before it exits) to the even CTA's
 // barriers; warps 3-18 are the softmax.  The even CTA's "full" barriers take
-// its own producer's arrival (with its bytes) and the relay; "P ready" and "O
-// read out" take one arrival per softmax warp of both CTAs; every completion
+// its own producer's arrival (with its bytes) and the relay; "P ready" (one
+// per score buffer) takes one arrival per warp of that buffer's softmax group
+// in both CTAs and "O read out" one per softmax warp of both CTAs; every completion
 // of products (S ready, PV done, stage and query buffers free) is committed
 // to the same barrier in both CTAs.  Every wait is bounded in time; both CTAs
 // meet at a cluster barrier before the tensor memory is released and before
@@ -56,19 +80,22 @@
 namespace pa {
 
 constexpr int kPairRowThreads = 4;                                   // softmax threads per query row
-constexpr int kPairRowScores = kUmmaTile / kPairRowThreads;          // scores per thread and token tile
+constexpr int kPairGroupRowThreads = kPairRowThreads / 2;            // per softmax group
+constexpr int kPairHalfScores = kUmmaTile / kPairGroupRowThreads;    // scores per thread and token tile (64)
 constexpr int kPairSoftmaxWarps = 4 * kPairRowThreads;               // four lane quarters
+constexpr int kPairGroupWarps = kPairSoftmaxWarps / 2;               // softmax warps per tile parity
 constexpr int kPairSoftmaxWarp0 = 3;                                  // first softmax warp
 constexpr int kPairThreads = 32 * (kPairSoftmaxWarp0 + kPairSoftmaxWarps);  // 608
 constexpr uint32_t kPairSBufCols = 128;                               // score buffer b at columns 128 b
-constexpr uint32_t kPairOCol = 256;                                   // O at columns 256 .. 256 + D - 1
+constexpr uint32_t kPairOCol = 256;                                   // O_b at columns 256 + 128 b ..
 constexpr int kPairRows = 2 * kUmmaRows;                              // query rows per cluster
 
 template <int D>
 __host__ __device__ constexpr size_t prefix_pair_layout_bytes(int stages) {
   return kSmemAlign + 2 * static_cast<size_t>(D / 64) * kUmmaRows * 128     // two query tiles
          + 2 * static_cast<size_t>(stages) * (D / 64) * kUmmaTile * 64       // K and V halves
-         + 2 * 2 * kUmmaRows * kPairRowThreads * sizeof(float)                    // maxima, sums
+         + 2 * 2 * kUmmaRows * kPairGroupRowThreads * sizeof(float)             // maxima [group][parity]
+         + 2 * kUmmaRows * kPairRowThreads * sizeof(float2)                    // (m, l) [segment parity]
          + (4 * static_cast<size_t>(stages) + 29) * sizeof(uint64_t) + 16;   // barriers, slots
 }
 
@@ -98,7 +125,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   constexpr uint32_t kVHalf = kUmmaTile * 128;           // V half per stage: one panel of 128 tokens (16 KB)
   constexpr uint32_t kQPanel = kUmmaRows * 128;          // one panel of Q (16 KB)
   constexpr uint32_t kQBytes = kHalves * kQPanel;        // one query tile
-  constexpr int kOQuart = D / kPairRowThreads;               // O columns per softmax thread
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr unsigned kFull = 0xffffffffu;
   constexpr uint16_t kBoth = 0x3;
@@ -111,9 +137,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   unsigned char* s_q = reinterpret_cast<unsigned char*>(base);          // [2][panel][128 rows][128 B]
   unsigned char* s_k = s_q + 2 * kQBytes;                                // [stage][panel][64 tok][128 B]
   unsigned char* s_v = s_k + static_cast<size_t>(stages) * kKHalf;      // [stage][128 tok][128 B]
-  float* x_max = reinterpret_cast<float*>(s_v + static_cast<size_t>(stages) * kVHalf);
-  float* s_sum = x_max + 2 * kUmmaRows * kPairRowThreads;
-  uint64_t* k_full = reinterpret_cast<uint64_t*>(s_sum + 2 * kUmmaRows * kPairRowThreads);
+  float* x_max = reinterpret_cast<float*>(s_v + static_cast<size_t>(stages) * kVHalf);   // [g][par][row][half]
+  float2* s_ml = reinterpret_cast<float2*>(x_max + 2 * 2 * kUmmaRows * kPairGroupRowThreads);  // [sb][row][4]
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(s_ml + 2 * kUmmaRows * kPairRowThreads);
   uint64_t* k_empty = k_full + stages;
   uint64_t* v_full = k_empty + stages;
   uint64_t* v_empty = v_full + stages;
@@ -124,7 +150,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* q_empty = q_full + 2;          // [2]
   uint64_t* o_free = q_empty + 2;          // (even CTA: both CTAs' softmax warps)
   uint64_t* drain = o_free + 1;
-  uint64_t* xq = drain + 1;                // [buffer][lane quarter]
+  uint64_t* xq = drain + 1;                // [group][lane quarter]
   uint64_t* sq = xq + 2 * 4;               // [segment parity][lane quarter]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sq + 2 * 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -148,7 +174,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 2 * kPairSoftmaxWarps);
+      mbar_init(&p_full[b], 2 * kPairGroupWarps);
       mbar_init(&pv_done[b], 1);
       mbar_init(&q_full[b], full_count);
       mbar_init(&q_empty[b], 1);
@@ -156,7 +182,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     mbar_init(o_free, 2 * kPairSoftmaxWarps);
     mbar_init(drain, 1);
     for (int i = 0; i < 2 * 4; ++i) {
-      mbar_init(&xq[i], kPairRowThreads);
+      mbar_init(&xq[i], kPairGroupRowThreads);
       mbar_init(&sq[i], kPairRowThreads);
     }
     *abort_flag = 0;
@@ -369,9 +395,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       auto issue_pv = [&](bool first) {
         const uint64_t vb = v_desc + ((vst * kVHalf) >> 4);
         const uint32_t a = tmem + static_cast<uint32_t>(tau_p & 1) * kPairSBufCols;
+        const uint32_t o = tmem + kPairOCol + static_cast<uint32_t>(tau_p & 1) * D;
 #pragma unroll
         for (int kk = 0; kk < kUmmaTile / 16; ++kk)
-          tc::mma_pair_ts(tmem + kPairOCol, a + 32 * (kk >> 1) + 8 * (kk & 1), vb + ((kk * 16 * 128) >> 4), idesc_o,
+          tc::mma_pair_ts(o, a + 32 * (kk >> 1) + 8 * (kk & 1), vb + ((kk * 16 * 128) >> 4), idesc_o,
                           !first || kk > 0);
         tc::commit_pair(&pv_done[tau_p & 1], kBoth);
         tc::commit_pair(&v_empty[vst], kBoth);
@@ -403,7 +430,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             break;
           }
           tc::fence_after_sync();
-          issue_pv(j == 0);
+          issue_pv(j < 2);
           if (j + 2 < n) {
             if (!issue_s(qb)) {
               ok = false;
@@ -419,18 +446,60 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
-    const int k = (warp - kPairSoftmaxWarp0) >> 2;             // column quarter
+    // Two groups of eight warps: group g takes the token tiles with tau mod 2
+    // = g (score buffer S_g, accumulator O_g) with its own reference maximum
+    // and sum, so one group's exponentials overlap the other's loads,
+    // exchanges and stores.  In a group two threads share a query row: half h
+    // takes scores 64 h .. 64 h + 63, 32 at a time.
+    const int sw = warp - kPairSoftmaxWarp0;
+    const int g = sw / kPairGroupWarps;                        // tile parity
+    const int half = (sw >> 2) & 1;                            // scores 64 half ..
     const int quarter = warp & 3;                              // tensor-memory lane quarter
     const int row = quarter * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t s_col = t_lane + static_cast<uint32_t>(g) * kPairSBufCols + half * kPairHalfScores;
+    const uint32_t og_col = t_lane + kPairOCol + static_cast<uint32_t>(g) * D + half * (D / 2);   // own half of O_g
+    const int cq = g * kPairGroupRowThreads + half;            // O columns 32 cq .. of the partial
     const float qk = prm.qk_scale;
     const float pad = qk >= 0.f ? -INFINITY : INFINITY;
     const float2 qk2 = make_float2(qk, qk);
-    const uint32_t lead_p_full = pair::map_shared(p_full, 0);
+    const uint32_t lead_p_full = pair::map_shared(&p_full[g], 0);
     const uint32_t lead_o_free = pair::map_shared(o_free, 0);
-    int tau = 0, items = 0;
-    bool ok = true;
-    auto weights = [&](uint32_t (&x)[32], float m_ref, int nq) {
+    // raw scores, chunk c of this half (columns 32 c ..), nq of them valid
+    auto load_chunk = [&](uint32_t (&x)[32], int c, int nq) {
+      tc::tmem_ld32(s_col + 32 * c, x);
+      tc::tmem_wait_ld();
+      if (nq < 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = j < nq ? x[j] : __float_as_uint(pad);
+      }
+    };
+    // largest (smallest, for a negative scale) raw score of x
+    auto chunk_ext = [&](const uint32_t (&x)[32]) {
+      float cm[4] = {__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]), __uint_as_float(x[3])};
+      if (qk >= 0.f) {
+#pragma unroll
+        for (int j = 4; j < 28; j += 8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cm[i] = fmax3(cm[i], __uint_as_float(x[j + i]), __uint_as_float(x[j + 4 + i]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cm[i] = fmaxf(cm[i], __uint_as_float(x[28 + i]));
+        return fmaxf(fmax3(cm[0], cm[1], cm[2]), cm[3]);
+      }
+#pragma unroll
+      for (int j = 4; j < 28; j += 8)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cm[i] = fmin3(cm[i], __uint_as_float(x[j + i]), __uint_as_float(x[j + 4 + i]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cm[i] = fminf(cm[i], __uint_as_float(x[28 + i]));
+      return fminf(fmin3(cm[0], cm[1], cm[2]), cm[3]);
+    };
+    // P = 2^(s * qk - m_ref) of the 32 scores in x rounded to T, two per
+    // column, into columns 32 c .. 32 c + 15 of this half (over the chunk's
+    // own scores); their sum before rounding into ls.  Of every 16
+    // exponentials kPolyExp are taken by the FMA-pipe polynomial; scores past
+    // the end of the tile get weight 0.
+    auto weights_store = [&](uint32_t (&x)[32], float m_ref, int nq, int c, float2 (&ls)[2]) {
       const float2 nm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -451,150 +520,151 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           x[16 * b + j + 1] = __float_as_uint(y.y);
         }
       }
-      if (nq < kPairRowScores) {
+      if (nq < 32) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = j < nq ? x[j] : 0u;
       }
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 e = make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+        w[i] = M::pack(e.x, e.y);
+        fadd2(ls[i & 1], e);
+      }
+      tc::tmem_st16(s_col + 32 * c, w);
     };
+    int tau = 0, items = 0;
+    bool ok = true;
     for (int u = u_begin; ok && u < u_end; ++items) {
       const PrefixSegment I = prefix_pair_segment<G>(u, u_end, prm);
       u = I.end;
+      const int tau0 = tau;
+      tau += I.ntiles;
       const int gr = I.row0 + static_cast<int>(rank) * kUmmaRows + row;
       const bool valid = gr < rows_total;
       const int s_idx = valid ? gr / G : 0;
       const int g_idx = valid ? gr - s_idx * G : 0;
       float m = -INFINITY, l = 0.f;
-      for (int t = 0; t < I.ntiles; ++t, ++tau) {
-        const int b = tau & 1;
-        const uint32_t ph = (tau >> 1) & 1;
+      const int t_first = (g - tau0) & 1;                      // this group's first tile of the segment
+      for (int t = t_first; t < I.ntiles; t += 2) {
+        const int tt = tau0 + t;
+        const uint32_t ph = (tt >> 1) & 1;                     // this group's tile count parity
         const int ntok = min(kUmmaTile, I.tok_hi - (I.tok_lo + t * kUmmaTile));
-        const int nq = min(kPairRowScores, max(0, ntok - k * kPairRowScores));
-        if (!__all_sync(kFull, mbar_wait(&s_full[b], ph, abort_flag))) {
+        const int nh = min(kPairHalfScores, max(0, ntok - half * kPairHalfScores));
+        const int nq0 = min(32, nh), nq1 = max(0, nh - 32);
+        if (!__all_sync(kFull, mbar_wait(&s_full[g], ph, abort_flag))) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t s_col = t_lane + static_cast<uint32_t>(b) * kPairSBufCols + k * kPairRowScores;
         uint32_t x[32];
-        tc::tmem_ld32(s_col, x);
-        tc::tmem_wait_ld();
-        if (nq < kPairRowScores) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = j < nq ? x[j] : __float_as_uint(pad);
-        }
-        float ext;
-        {
-          float cm[4] = {__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]), __uint_as_float(x[3])};
-          if (qk >= 0.f) {
-#pragma unroll
-            for (int j = 4; j < 28; j += 8)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) cm[i] = fmax3(cm[i], __uint_as_float(x[j + i]), __uint_as_float(x[j + 4 + i]));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cm[i] = fmaxf(cm[i], __uint_as_float(x[28 + i]));
-            ext = fmaxf(fmax3(cm[0], cm[1], cm[2]), cm[3]);
-          } else {
-#pragma unroll
-            for (int j = 4; j < 28; j += 8)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) cm[i] = fmin3(cm[i], __uint_as_float(x[j + i]), __uint_as_float(x[j + 4 + i]));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cm[i] = fminf(cm[i], __uint_as_float(x[28 + i]));
-            ext = fminf(fmin3(cm[0], cm[1], cm[2]), cm[3]);
-          }
-        }
-        x_max[(b * kUmmaRows + row) * kPairRowThreads + k] = nq > 0 ? ext * qk : -INFINITY;
+        load_chunk(x, 0, nq0);
+        const float e0 = chunk_ext(x);
+        load_chunk(x, 1, nq1);                                 // x holds chunk 1 from here
+        const float e1 = chunk_ext(x);
+        const float ext = qk >= 0.f ? fmaxf(e0, e1) : fminf(e0, e1);
+        const float c_own = nh > 0 ? ext * qk : -INFINITY;
+        float* slot = x_max + ((g * 2 + static_cast<int>(ph)) * kUmmaRows + row) * kPairGroupRowThreads;
+        slot[half] = c_own;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&xq[b * 4 + quarter]);
-        const bool spec = __all_sync(kFull, m != -INFINITY);
-        if (spec) weights(x, m, nq);
-        if (!__all_sync(kFull, mbar_wait(&xq[b * 4 + quarter], ph, abort_flag))) {
+        if (lane == 0) mbar_arrive(&xq[g * 4 + quarter]);
+        if (!__all_sync(kFull, mbar_wait(&xq[g * 4 + quarter], ph, abort_flag))) {
           ok = false;
           break;
         }
-        const float4 c4 = *reinterpret_cast<const float4*>(x_max + (b * kUmmaRows + row) * kPairRowThreads);
-        const float c = fmaxf(fmaxf(c4.x, c4.y), fmaxf(c4.z, c4.w));
+        const float c = fmaxf(c_own, slot[half ^ 1]);
         const bool need = c > m + kTau;
         if (__any_sync(kFull, need)) {
           const float mn = need ? c : m;
-          const float f = mn != m ? exp2_approx(m - mn) : 1.f;
-          if (t >= 1) {
-            if (!__all_sync(kFull, mbar_wait(&pv_done[(tau - 1) & 1], ((tau - 1) >> 1) & 1, abort_flag))) {
+          const float f = mn != m ? exp2_approx(m - mn) : 1.f;     // 0 when m was -inf
+          if (t >= 2) {
+            // O_g holds the group's earlier products of the segment once
+            // PV(tt - 2) has completed; this thread's half of O_g
+            if (!__all_sync(kFull, mbar_wait(&pv_done[g], ((tt - 2) >> 1) & 1, abort_flag))) {
               ok = false;
               break;
             }
             tc::fence_after_sync();
-            uint32_t o[32];
-            tc::tmem_ld32(t_lane + kPairOCol + k * kOQuart, o);
-            tc::tmem_wait_ld();
+#pragma unroll 1
+            for (int ob = 0; ob < 4; ++ob) {
+              uint32_t o[16];
+              tc::tmem_ld16(og_col + ob * 16, o);
+              tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-            tc::tmem_st32(t_lane + kPairOCol + k * kOQuart, o);
+              for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+              tc::tmem_st16(og_col + ob * 16, o);
+            }
           }
           l *= f;
           m = mn;
-          if (spec) {
-            tc::tmem_ld32(s_col, x);
-            tc::tmem_wait_ld();
-          }
-          weights(x, m, nq);
         }
+        // chunk 1 from the registers first (its weights overwrite only its own
+        // scores), then chunk 0 again from tensor memory
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 e = make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
-          w[i] = M::pack(e.x, e.y);
-          fadd2(ls[i & 1], e);
-        }
-        tc::tmem_st16(s_col, w);
+        weights_store(x, m, nq1, 1, ls);
+        load_chunk(x, 0, nq0);
+        weights_store(x, m, nq0, 0, ls);
         tc::tmem_wait_st();
         l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) {
-          if (lead) mbar_arrive(&p_full[b]);
-          else pair::arrive_cluster(lead_p_full + b * 8);
+          if (lead) mbar_arrive(&p_full[g]);
+          else pair::arrive_cluster(lead_p_full);
         }
       }
       if (!ok) break;
       if (I.ntiles > 0) {
+        // the segment's last product has completed: O_0 and O_1 are final
         if (!__all_sync(kFull, mbar_wait(&pv_done[(tau - 1) & 1], ((tau - 1) >> 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
       }
+      // the row's (m, l) of both groups: O = 2^(m_0 - M) O_0 + 2^(m_1 - M) O_1
       const int sb = items & 1;
-      s_sum[(sb * kUmmaRows + row) * kPairRowThreads + k] = l;
+      float2* ml = s_ml + (sb * kUmmaRows + row) * kPairRowThreads;
+      ml[cq] = make_float2(m, l);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sq[sb * 4 + quarter]);
       if (!__all_sync(kFull, mbar_wait(&sq[sb * 4 + quarter], (items >> 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
-      const float4 l4 = *reinterpret_cast<const float4*>(s_sum + (sb * kUmmaRows + row) * kPairRowThreads);
-      const float l_row = (l4.x + l4.y) + (l4.z + l4.w);
+      const float4 a01 = *reinterpret_cast<const float4*>(ml);
+      const float4 a23 = *reinterpret_cast<const float4*>(ml + 2);
+      const bool has0 = I.ntiles > ((0 - tau0) & 1), has1 = I.ntiles > ((1 - tau0) & 1);
+      const float m0 = a01.x, l0 = a01.y + a01.w, m1 = a23.x, l1 = a23.y + a23.w;
+      const float mx = fmaxf(has0 ? m0 : -INFINITY, has1 ? m1 : -INFINITY);
+      const float f0 = has0 ? exp2_approx(m0 - mx) : 0.f;
+      const float f1 = has1 ? exp2_approx(m1 - mx) : 0.f;
       const size_t pi = (static_cast<size_t>(s_idx) * prm.num_q_heads + I.h * G + g_idx) * prm.max_parts + I.split0;
-      float* dst = prm.part_acc + pi * D + k * kOQuart;
-      uint32_t o[kOQuart];
-      if (I.ntiles > 0) {
-        tc::tmem_ld32(t_lane + kPairOCol + k * kOQuart, o);
+      float* dst = prm.part_acc + pi * D + cq * 32;
+      const uint32_t o0_col = t_lane + kPairOCol + cq * 32, o1_col = o0_col + D;
+#pragma unroll 1
+      for (int ob = 0; ob < 2; ++ob) {
+        uint32_t a0[16], a1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) a0[j] = a1[j] = 0u;
+        if (has0) tc::tmem_ld16(o0_col + ob * 16, a0);
+        if (has1) tc::tmem_ld16(o1_col + ob * 16, a1);
         tc::tmem_wait_ld();
-      } else {
 #pragma unroll
-        for (int j = 0; j < kOQuart; ++j) o[j] = 0u;
-      }
-      if (valid) {
+        for (int j = 0; j < 16; ++j)
+          a0[j] = __float_as_uint(f0 * __uint_as_float(a0[j]) + f1 * __uint_as_float(a1[j]));
+        if (valid) {
 #pragma unroll
-        for (int j = 0; j < kOQuart; j += 4)
-          *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]),
-                                                            __uint_as_float(o[j + 2]), __uint_as_float(o[j + 3]));
-        if (k == 0) {
-          prm.part_ml[pi] = make_float2(m, l_row);
-          for (int sp = 1; sp < I.split1 - I.split0; ++sp) prm.part_ml[pi + sp] = make_float2(-INFINITY, 0.f);
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + ob * 16 + j) = make_float4(
+                __uint_as_float(a0[j]), __uint_as_float(a0[j + 1]), __uint_as_float(a0[j + 2]), __uint_as_float(a0[j + 3]));
         }
       }
+      if (valid && cq == 0) {
+        prm.part_ml[pi] = make_float2(mx, f0 * l0 + f1 * l1);
+        for (int sp = 1; sp < I.split1 - I.split0; ++sp) prm.part_ml[pi + sp] = make_float2(-INFINITY, 0.f);
+      }
+      // O_0 and O_1 have been read out: the next segment's first products may overwrite them
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) {
