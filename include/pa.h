@@ -263,7 +263,7 @@ pa_status pa_decode_attention(const void* q, const void* k_cache, const void* v_
  * bytes for the work-unit counter, the suffix's work-unit list (as for
  * pa_decode_workspace_size) and one float32 partial (max, sum, D values) per
  * (sequence, query head, part), where the parts are the prefix's
- * ceil(prefix_len / 1024) slices followed by the suffix's partitions
+ * ceil(prefix_len / 512) slices followed by the suffix's partitions
  * (ceil(max_suffix_blocks * block_size / partition_size), or 1 when
  * partition_size == 0).  0 for invalid sizes. */
 size_t pa_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
@@ -277,8 +277,17 @@ size_t pa_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
  * block table prefix_blocks ++ suffix_tables[s] and context length
  * prefix_len + suffix_lens[s].  The prefix is attended once per KV head for
  * all S*G query rows together on the tensor cores (each prefix K/V tile read
- * once per 64 query rows), the suffixes by the decode kernel, and one merge
+ * once per 256 query rows), the suffixes by the decode kernel, and one merge
  * combines the partial results.
+ *
+ * Streams: the prefix kernel runs on a side stream of the library's (one per
+ * device, created on first use, highest priority), forked from `stream` by
+ * an event and joined back to it before the merge, so that the suffixes'
+ * planner and decode on `stream` may run at the same time.  All the call's
+ * work follows what was queued on `stream` before it and precedes what is
+ * queued after it; the side stream also orders the prefix kernels of calls
+ * on different streams.  With PA_PREFIX_SERIAL=1 in the environment every
+ * kernel runs on `stream`, one after the other.
  *
  *   prefix_blocks  device int32 [prefix_len / block_size]
  *   prefix_len     tokens; a multiple of block_size and of 16 (0: plain call)

@@ -100,6 +100,7 @@ struct DecodeArgs {
   int table_stride = 0;          // 0: rows of block_tables are max_blocks apart
   int part_offset = 0;           // partials before partition 0 (prefix splits)
   int total_parts = 0;           // 0: ceil(max_blocks*block_size/P), else the partial row stride
+  cudaEvent_t merge_after = nullptr;  // the merge also waits for this event (the prefix kernel's side stream)
 };
 
 constexpr size_t kSchedBytes = 256;   // unit counter and unit count at the head of the workspace
@@ -333,6 +334,12 @@ pa_status launch_decode(const DecodeArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (a.merge_after) {
+      // the join with the side stream: an ordinary launch after the event
+      e = cudaStreamWaitEvent(a.stream, a.merge_after, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent(merge after the prefix kernel)");
+      cfg.numAttrs = 0;
+    }
     // six rows a warp in flight where a head has more than 16 partitions (one
     // round of loads for up to 48 partitions; 64 registers, so a 70B-shaped
     // merge of 512 CTAs is one wave), four otherwise (48 registers)

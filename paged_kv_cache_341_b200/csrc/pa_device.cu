@@ -295,6 +295,35 @@ pa_status dispatch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   }
 }
 
+// The shared-prefix call's side stream on each device (created on first use,
+// highest priority) and the events of its fork and join.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;              // one call's fork, launches and join at a time
+};
+
+pa_status side_stream(SideStream** out) {
+  static std::mutex mu;
+  static SideStream cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= 64) return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: device index above 63");
+  std::lock_guard<std::mutex> lock(mu);
+  SideStream& s = cache[dev];
+  if (!s.stream) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&s.stream, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "shared prefix: side stream and events");
+  }
+  *out = &s;
+  return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -538,8 +567,31 @@ pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, 
   a.part_offset = prefix_splits(prefix_len);
   a.total_parts = a.part_offset + max_parts(max_suffix_blocks, block_size, partition_size);
   const PrefixArgs pf{prefix_blocks, prefix_len};
-  pa_status st = dtype == PA_F16 ? dispatch_prefix<__half>(a, pf) : dispatch_prefix<__nv_bfloat16>(a, pf);
+  if (env_int("PA_PREFIX_SERIAL")) {
+    // everything on the caller's stream, one kernel after the other
+    pa_status st = dtype == PA_F16 ? dispatch_prefix<__half>(a, pf) : dispatch_prefix<__nv_bfloat16>(a, pf);
+    if (st != PA_OK) return st;
+    st = dtype == PA_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+    return st == PA_OK ? pa::ok() : st;
+  }
+  // The prefix kernel on a side stream forked from the caller's; the
+  // suffixes' planner and decode on the caller's stream meanwhile; the merge
+  // after both (the side stream joins before it).  The two halves share no
+  // data until the merge, so they may run in either order or together.
+  SideStream* ss = nullptr;
+  pa_status st = side_stream(&ss);
   if (st != PA_OK) return st;
+  std::lock_guard<std::mutex> lock(ss->mu);
+  cudaError_t e = cudaEventRecord(ss->fork, a.stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "shared prefix: fork to the side stream");
+  DecodeArgs ap = a;
+  ap.stream = ss->stream;
+  st = dtype == PA_F16 ? dispatch_prefix<__half>(ap, pf) : dispatch_prefix<__nv_bfloat16>(ap, pf);
+  if (st != PA_OK) return st;
+  e = cudaEventRecord(ss->join, ss->stream);
+  if (e != cudaSuccess) return cuda_fail(e, "shared prefix: join event");
+  a.merge_after = ss->join;
   st = dtype == PA_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
   return st == PA_OK ? pa::ok() : st;
 }

@@ -34,7 +34,9 @@ def prefix_path(request, monkeypatch):
     return request.param
 
 
-def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed, q_scale=1.0):
+def cascade_case(dtype, hkv, d, bs, prefix_len, suffixes, seed):
+    """A pool whose sequences share prefix_len tokens copy-on-write, then hold
+    their own suffixes; returns the cache and its host K/V contents."""
     from paged_kv_cache_341_b200.cache import PagedKVCache
     rng = np.random.default_rng(seed)
     s = len(suffixes)
@@ -55,6 +57,13 @@ def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed
     cache.k_cache.copy_(k_host)
     cache.v_cache.copy_(v_host)
     cache.upload_tables()
+    return cache, k_host, v_host, mb
+
+
+def run_cascade(pa, dtype, hq, hkv, d, bs, prefix_len, suffixes, partition, seed, q_scale=1.0):
+    s = len(suffixes)
+    pblocks = prefix_len // bs
+    cache, k_host, v_host, mb = cascade_case(dtype, hkv, d, bs, prefix_len, suffixes, seed)
     q_host = workloads.randn((s, hq, d), dtype, seed + 2)
     if q_scale != 1.0:
         q_host = (q_host.float() * q_scale).to(TORCH[dtype])
@@ -123,6 +132,45 @@ def test_large_scores_rescale_in_tensor_memory(pa, prefix_path):
     gpu, ref, _ = run_cascade(pa, "bf16", 16, 4, 128, 16, 1024 + 512, [3, 0, 40], 0, seed=8, q_scale=12.0)
     check_launched(pa, prefix_path, 128)
     assert_close(gpu, ref, "bf16", "large scores")
+
+
+def test_back_to_back_calls_on_a_stream(pa, prefix_path):
+    # The prefix kernel runs on the library's side stream, forked from the
+    # caller's stream and joined back before the merge.  Three calls queued on
+    # a non-default stream without a sync, sharing one workspace, each with
+    # queries written on that stream just before it: every output must be its
+    # own call's.
+    dtype, hq, hkv, d, bs, prefix_len = "bf16", 32, 8, 128, 16, 2048 + 64
+    rng = np.random.default_rng(11)
+    suffixes = [int(x) for x in rng.integers(0, 300, size=40)]
+    s, pblocks = len(suffixes), prefix_len // bs
+    cache, k_host, v_host, _ = cascade_case(dtype, hkv, d, bs, prefix_len, suffixes, 12)
+    scale = 1.0 / math.sqrt(d)
+    prefix_ids = cache.d_tables[0, :pblocks].contiguous()
+    suffix_tables = cache.d_tables[:, pblocks:]
+    suffix_lens = (cache.d_lens - prefix_len).contiguous()
+    q_hosts = [workloads.randn((s, hq, d), dtype, 20 + i) for i in range(3)]
+    q_srcs = [q.cuda() for q in q_hosts]
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    ws = None
+    outs = []
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            q_i = torch.empty_like(q_srcs[i])
+            q_i.copy_(q_srcs[i])          # written on the stream right before the call
+            out = torch.full((s, hq, d), float("nan"), dtype=TORCH[dtype], device="cuda")
+            ws = pa.pa_decode_attention_shared_prefix(q_i, cache.k_cache, cache.v_cache, prefix_ids, prefix_len,
+                                                      suffix_tables, suffix_lens, scale, out, partition_size=512,
+                                                      workspace=ws, stream=stream)
+            outs.append(out)
+    stream.synchronize()
+    assert pa.pa_device_error() == 0
+    check_launched(pa, prefix_path, d)
+    for i in range(3):
+        ref = oracle_decode(q_hosts[i].double().numpy(), AsF64(k_host), AsF64(v_host),
+                            [list(r) for r in cache.tables], [int(x) for x in cache.lens], scale)
+        assert_close(outs[i].float().cpu().numpy(), ref, dtype, "%s call %d" % (prefix_path, i))
 
 
 def test_zero_prefix_is_the_plain_call(pa):
