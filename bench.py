@@ -76,8 +76,8 @@ def call_label(cascade, w, batch, calls, peak_kind):
     # the one-warp planner serves batches of up to 32 sequences
     planner = "plan_small_kernel" if batch <= 32 else "plan_kernel"
     if cascade:
-        prefix = {"mma": "prefix_attention_kernel", "pair": "prefix_pair_kernel"}.get(
-            os.environ.get("PA_PREFIX_PATH", ""), "prefix_umma_kernel")
+        prefix = {"mma": "prefix_attention_kernel", "umma": "prefix_umma_kernel"}.get(
+            os.environ.get("PA_PREFIX_PATH", ""), "prefix_pair_kernel")
         return ("pa_decode_attention_shared_prefix call (%s + %s + %s + reduce_kernel), median of %d "
                 "calls; achieved counts the logical K/V bytes of every sequence (the shared prefix once per "
                 "sequence), so a frac above 1 measures the sharing, not HBM; peak = %s copy bandwidth"

@@ -449,10 +449,10 @@ pa_status pa_debug_decode_stall(int64_t wait_limit_ns);
 /* Which kernel the last pa_decode_attention_shared_prefix call of this
  * thread launched for the prefix: 1 = the SM-pair tensor-core kernel (two-CTA
  * clusters, head_dim 128), 2 = the one-SM tensor-core kernel, 3 = the
- * mma.sync kernel, 0 = none yet.  The one-SM kernel is the default;
- * PA_PREFIX_PATH=pair in the environment picks the SM-pair kernel (which
+ * mma.sync kernel, 0 = none yet.  The SM-pair kernel is the default (it
  * falls back to the one-SM kernel for head_dim 64 or when no cluster of two
- * is resident) and PA_PREFIX_PATH=mma the mma.sync kernel.  A test and
+ * is resident); PA_PREFIX_PATH=umma in the environment picks the one-SM
+ * kernel and PA_PREFIX_PATH=mma the mma.sync kernel.  A test and
  * measurement aid: returns the value, never fails. */
 int pa_debug_last_prefix_kernel(void);
 

@@ -34,17 +34,17 @@ struct PrefixArgs {
   int prefix_len;
 };
 
-// Prefix kernel: the one-SM tcgen05 kernel by default; PA_PREFIX_PATH=pair
-// picks the SM-pair tcgen05 kernel (head_dim 128, where clusters of two fit;
-// else the default) and PA_PREFIX_PATH=mma the mma.sync kernel (same results
-// within rounding, kept for comparison).
+// Prefix kernel: the SM-pair tcgen05 kernel by default (head_dim 128, where
+// clusters of two fit; else the one-SM tcgen05 kernel); PA_PREFIX_PATH=umma
+// picks the one-SM kernel and PA_PREFIX_PATH=mma the mma.sync kernel (same
+// results within rounding, kept for comparison).
 enum class PrefixPath { kUmma, kPair, kMma };
 thread_local int g_last_prefix_kernel = 0;     // pa_debug_last_prefix_kernel
 PrefixPath prefix_path() {
   const char* v = std::getenv("PA_PREFIX_PATH");
   if (v && std::string(v) == "mma") return PrefixPath::kMma;
-  if (v && std::string(v) == "pair") return PrefixPath::kPair;
-  return PrefixPath::kUmma;
+  if (v && std::string(v) == "umma") return PrefixPath::kUmma;
+  return PrefixPath::kPair;
 }
 
 // Queries [S][Hq][D] as a 4-D map (64 elements, D / 64 panels, Hq heads, S

@@ -1,5 +1,7 @@
 // Shared-prefix ("cascade") decode, prefix half, on the fifth-generation
-// tensor cores (tcgen05 + tensor memory), sm_100a.
+// tensor cores (tcgen05 + tensor memory), sm_100a: the one-SM form, used for
+// head_dim 64, where no cluster of two CTAs fits, and with
+// PA_PREFIX_PATH=umma (the SM-pair form in prefix_tc2.cuh is the default).
 //
 // Same contract as prefix_attention_kernel: for one KV head h, up to two
 // tiles of 128 query rows (of the S*G rows that use head h) and one slice of

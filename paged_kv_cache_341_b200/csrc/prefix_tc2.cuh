@@ -1,8 +1,9 @@
 // Shared-prefix ("cascade") decode, prefix half, on the tensor cores of an
 // SM pair (tcgen05 cta_group::2, clusters of two CTAs), sm_100a, D = 128.
 //
-// Same contract as prefix_umma_kernel (the one-SM form in prefix_tc.cuh, the
-// default; this one is chosen with PA_PREFIX_PATH=pair): attention over the shared
+// Same contract as prefix_umma_kernel (the one-SM form in prefix_tc.cuh, used
+// for head_dim 64, when no cluster of two fits, or with PA_PREFIX_PATH=umma;
+// this kernel is the default for head_dim 128): attention over the shared
 // prefix is one dense product per KV head once the rows of every sequence are
 // stacked ("Paged Attention", aidolsgroup.com, "Example"; prefixes shared
 // copy-on-write, agentechip.com "Shared Prefix Caching").  What the pair
@@ -35,10 +36,16 @@
 // exchange (m, l) and each writes a quarter of the partial,
 // 2^(m_0 - M) O_0 + 2^(m_1 - M) O_1 with M = max(m_0, m_1).
 //
-// Measured on the 200-sequence, 30,720-token shared-prefix step (B200): a
-// cascade call of 0.2253 ms against 0.2262 ms with the one-SM kernel on the
-// same box (with one softmax group of sixteen warps over both score buffers:
-// 0.231 against 0.225 ms).  Clock stamps per tile show each group busy
+// K and V halves of a stage share one "full" barrier (both producers arrive
+// with their bytes; in the even CTA the relay passes on both of the odd CTA's)
+// and one "empty" barrier, committed after the stage's PV: one wait and one
+// commit per tile fewer for the issuing thread, which sets the period.
+//
+// Measured on the 200-sequence, 30,720-token shared-prefix step (B200), with
+// every kernel on one stream: a cascade call of 0.2182 ms against 0.2245 ms
+// with the one-SM kernel on the same box (separate K and V barriers: 0.2243;
+// one softmax group of sixteen warps over both score buffers: 0.231 against
+// 0.225 ms).  Clock stamps per tile show each group busy
 // ~2.2K of its ~4.5K-cycle period (loads and maximum ~440, exchange ~300,
 // exponentials and stores ~1.3K) and the issuing thread spending ~1.3K cycles
 // per tile in the sixteen M 256 x N 128 x K 16 products (about 80-87 cycles
@@ -139,11 +146,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   unsigned char* s_v = s_k + static_cast<size_t>(stages) * kKHalf;      // [stage][128 tok][128 B]
   float* x_max = reinterpret_cast<float*>(s_v + static_cast<size_t>(stages) * kVHalf);   // [g][par][row][half]
   float2* s_ml = reinterpret_cast<float2*>(x_max + 2 * 2 * kUmmaRows * kPairGroupRowThreads);  // [sb][row][4]
+  // K and V of a stage share one "full" and one "empty" barrier
   uint64_t* k_full = reinterpret_cast<uint64_t*>(s_ml + 2 * kUmmaRows * kPairRowThreads);
   uint64_t* k_empty = k_full + stages;
-  uint64_t* v_full = k_empty + stages;
-  uint64_t* v_empty = v_full + stages;
-  uint64_t* s_full = v_empty + stages;     // [2]
+  uint64_t* v_full = k_full;
+  uint64_t* v_empty = k_empty;
+  uint64_t* s_full = k_empty + 3 * stages;     // [2]
   uint64_t* p_full = s_full + 2;           // [2] (even CTA: both CTAs' softmax warps)
   uint64_t* pv_done = p_full + 2;          // [2]
   uint64_t* q_full = pv_done + 2;          // [2]
@@ -165,12 +173,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int u_end = static_cast<int>(static_cast<long long>(cluster + 1) * prm.num_units / clusters);
 
   if (threadIdx.x == 0) {
-    const uint32_t full_count = lead ? 2 : 1;     // even CTA: own producer + the odd CTA's relay
+    // even CTA: own two producers + the odd CTA's relay of each
+    const uint32_t full_count = lead ? 2 : 1;
     for (int i = 0; i < stages; ++i) {
-      mbar_init(&k_full[i], full_count);
+      mbar_init(&k_full[i], 2 * full_count);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], full_count);
-      mbar_init(&v_empty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -384,7 +391,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tc::mma_pair_ss(d, qbd + (((kk >> 2) * kQPanel + (kk & 3) * 32) >> 4),
                           kb + (((kk >> 2) * kKPanel + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
         tc::commit_pair(&s_full[tau_s & 1], kBoth);
-        tc::commit_pair(&k_empty[kst], kBoth);
         if (++kst == stages) {
           kst = 0;
           kph ^= 1;
@@ -423,8 +429,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (!ok) break;
         if (n <= 2) tc::commit_pair(&q_empty[qb], kBoth);
         for (int j = 0; j < n; ++j) {
-          if (!mbar_wait(&v_full[vst], vph, abort_flag) ||
-              !mbar_wait(&p_full[tau_p & 1], (tau_p >> 1) & 1, abort_flag) ||
+          // V of this tile landed with its K, which S waited for
+          if (!mbar_wait(&p_full[tau_p & 1], (tau_p >> 1) & 1, abort_flag) ||
               (j == 0 && items > 0 && !mbar_wait(o_free, (items - 1) & 1, abort_flag))) {
             ok = false;
             break;

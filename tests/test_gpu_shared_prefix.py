@@ -28,8 +28,8 @@ def pa():
 
 @pytest.fixture(params=["umma", "pair", "mma"])
 def prefix_path(request, monkeypatch):
-    """Run a test on each prefix kernel: the one-SM tcgen05 kernel (the default), the SM-pair tcgen05
-    kernel (head_dim 128; 64 falls back to the one-SM kernel) and the mma.sync one."""
+    """Run a test on each prefix kernel: the SM-pair tcgen05 kernel (the default for head_dim 128; 64
+    falls back to the one-SM kernel), the one-SM tcgen05 kernel and the mma.sync one."""
     monkeypatch.setenv("PA_PREFIX_PATH", request.param)
     return request.param
 

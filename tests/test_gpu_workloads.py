@@ -141,17 +141,18 @@ def test_full_size_step(name):
     assert_close(out.float().cpu().numpy(), ref, w.dtype, "%s, every (sequence, head)" % name)
 
 
-def test_shared_prefix_full_size_step_plain_and_cascade(monkeypatch):
+@pytest.mark.parametrize("prefix_path", ["pair", "umma"])
+def test_shared_prefix_full_size_step_plain_and_cascade(monkeypatch, prefix_path):
     """The shared-prefix step: copy-on-write of the forks' partly filled last blocks, append,
     then attention twice over the same state -- the plain partitioned call and the cascade
-    call (prefix once for all 200 x 32 query rows on the tcgen05 kernel, 30 slices of 1,024
-    tokens, suffix partitions of 512, merge)."""
+    call (prefix once for all 200 x 32 query rows on a tcgen05 kernel -- the SM-pair one, the
+    default, or the one-SM one -- 60 slices of 512 tokens, suffix partitions of 512, merge)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from paged_kv_cache_341_b200 import pa
     sc, q, q_dev, plain, btables, blens = full_step("shared_prefix")
     w, c = sc.w, sc.cache
-    monkeypatch.setenv("PA_PREFIX_PATH", "umma")
+    monkeypatch.setenv("PA_PREFIX_PATH", prefix_path)
     pblocks = w.shared_prefix // w.block_size
     prefix_ids = c.d_tables[sc.rows.start, :pblocks].contiguous()
     suffix_tables = c.d_tables[sc.rows, pblocks:]
@@ -164,6 +165,7 @@ def test_shared_prefix_full_size_step_plain_and_cascade(monkeypatch):
                                          suffix_lens, w.scale, casc, w.partition_size, ws)
     torch.cuda.synchronize()
     assert pa.pa_device_error() == 0
+    assert pa.pa_debug_last_prefix_kernel() == {"pair": 1, "umma": 2}[prefix_path]
     for r in range(sc.batch):
         assert btables[r][:pblocks] == btables[0][:pblocks]
     plain_h = plain.float().cpu().numpy()
