@@ -38,14 +38,17 @@
 //
 // K and V halves of a stage share one "full" barrier (both producers arrive
 // with their bytes; in the even CTA the relay passes on both of the odd CTA's)
-// and one "empty" barrier, committed after the stage's PV: one wait and one
-// commit per tile fewer for the issuing thread, which sets the period.
+// and one "empty" barrier, committed after the stage's PV, which is also how
+// the softmax learns that PV(t) has completed (the empty phase of tile t's
+// stage): per tile the issuing thread, which sets the period, waits twice
+// (K and V, the weights) and commits twice (S ready, stage free).
 //
 // Measured on the 200-sequence, 30,720-token shared-prefix step (B200), with
-// every kernel on one stream: a cascade call of 0.2182 ms against 0.2245 ms
-// with the one-SM kernel on the same box (separate K and V barriers: 0.2243;
-// one softmax group of sixteen warps over both score buffers: 0.231 against
-// 0.225 ms).  Clock stamps per tile show each group busy
+// every kernel on one stream: a cascade call of 0.2189 ms against 0.2221 ms
+// with a separate "PV done" commit; with that commit, 0.2182 against 0.2245 ms
+// for the one-SM kernel on one box, and 0.2243 ms with separate K and V
+// barriers too (one softmax group of sixteen warps over both score buffers:
+// 0.231 against 0.225 ms).  Clock stamps per tile show each group busy
 // ~2.2K of its ~4.5K-cycle period (loads and maximum ~440, exchange ~300,
 // exponentials and stores ~1.3K) and the issuing thread spending ~1.3K cycles
 // per tile in the sixteen M 256 x N 128 x K 16 products (about 80-87 cycles
@@ -70,7 +73,7 @@
 // its own producer's arrival (with its bytes) and the relay; "P ready" (one
 // per score buffer) takes one arrival per warp of that buffer's softmax group
 // in both CTAs and "O read out" one per softmax warp of both CTAs; every completion
-// of products (S ready, PV done, stage and query buffers free) is committed
+// of products (S ready, stage and query buffers free) is committed
 // to the same barrier in both CTAs.  Every wait is bounded in time; both CTAs
 // meet at a cluster barrier before the tensor memory is released and before
 // either exits, so no copy or product still touches a CTA that has gone.
@@ -153,8 +156,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* v_empty = k_empty;
   uint64_t* s_full = k_empty + 3 * stages;     // [2]
   uint64_t* p_full = s_full + 2;           // [2] (even CTA: both CTAs' softmax warps)
-  uint64_t* pv_done = p_full + 2;          // [2]
-  uint64_t* q_full = pv_done + 2;          // [2]
+  // PV(t) completion is the "empty" phase of tile t's stage
+  uint64_t* q_full = p_full + 4;           // [2]
   uint64_t* q_empty = q_full + 2;          // [2]
   uint64_t* o_free = q_empty + 2;          // (even CTA: both CTAs' softmax warps)
   uint64_t* drain = o_free + 1;
@@ -182,7 +185,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 2 * kPairGroupWarps);
-      mbar_init(&pv_done[b], 1);
       mbar_init(&q_full[b], full_count);
       mbar_init(&q_empty[b], 1);
     }
@@ -406,7 +408,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kk = 0; kk < kUmmaTile / 16; ++kk)
           tc::mma_pair_ts(o, a + 32 * (kk >> 1) + 8 * (kk & 1), vb + ((kk * 16 * 128) >> 4), idesc_o,
                           !first || kk > 0);
-        tc::commit_pair(&pv_done[tau_p & 1], kBoth);
         tc::commit_pair(&v_empty[vst], kBoth);
         if (++vst == stages) {
           vst = 0;
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (t >= 2) {
             // O_g holds the group's earlier products of the segment once
             // PV(tt - 2) has completed; this thread's half of O_g
-            if (!__all_sync(kFull, mbar_wait(&pv_done[g], ((tt - 2) >> 1) & 1, abort_flag))) {
+            if (!__all_sync(kFull, mbar_wait(&k_empty[(tt - 2) % stages], ((tt - 2) / stages) & 1, abort_flag))) {
               ok = false;
               break;
             }
@@ -622,7 +623,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (!ok) break;
       if (I.ntiles > 0) {
         // the segment's last product has completed: O_0 and O_1 are final
-        if (!__all_sync(kFull, mbar_wait(&pv_done[(tau - 1) & 1], ((tau - 1) >> 1) & 1, abort_flag))) {
+        if (!__all_sync(kFull, mbar_wait(&k_empty[(tau - 1) % stages], ((tau - 1) / stages) & 1, abort_flag))) {
           ok = false;
           break;
         }
