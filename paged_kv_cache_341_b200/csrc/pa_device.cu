@@ -295,11 +295,32 @@ pa_status dispatch_prefix(const DecodeArgs& a, const PrefixArgs& pf) {
   }
 }
 
+// The driver context current on this thread (nullptr before the thread's
+// first runtime call binds one).
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
 // The shared-prefix call's side stream on each device (created on first use,
-// highest priority) and the events of its fork and join.
+// highest priority) and the events of its fork and join.  They belong to the
+// context they were made in: another context on the device (after a device
+// reset, or one the caller bound) gets its own.
 struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  CUcontext ctx = nullptr;
   std::mutex mu;              // one call's fork, launches and join at a time
 };
 
@@ -312,13 +333,20 @@ pa_status side_stream(SideStream** out) {
   if (dev >= 64) return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: device index above 63");
   std::lock_guard<std::mutex> lock(mu);
   SideStream& s = cache[dev];
-  if (!s.stream) {
+  const CUcontext ctx = current_context();
+  if (!s.stream || (ctx && s.ctx && ctx != s.ctx)) {
+    // (the handles of a context that is gone are dropped, not destroyed)
     int least = 0, greatest = 0;
+    s.stream = nullptr;
     e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&s.stream, cudaStreamNonBlocking, greatest);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) return cuda_fail(e, "shared prefix: side stream and events");
+    if (e != cudaSuccess) {
+      s.stream = nullptr;
+      return cuda_fail(e, "shared prefix: side stream and events");
+    }
+    s.ctx = current_context();
   }
   *out = &s;
   return PA_OK;
