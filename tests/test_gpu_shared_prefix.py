@@ -173,6 +173,58 @@ def test_back_to_back_calls_on_a_stream(pa, prefix_path):
         assert_close(outs[i].float().cpu().numpy(), ref, dtype, "%s call %d" % (prefix_path, i))
 
 
+def test_calls_from_two_host_threads(pa):
+    # Two host threads, each with its own stream, workspace and queries, call
+    # the cascade at the same time; the library's side stream (and its fork and
+    # join events) is shared, so each call's fork, prefix launch and join must
+    # stay together.  Every output must be its own call's.
+    import threading
+    dtype, hq, hkv, d, bs, prefix_len = "bf16", 16, 4, 128, 16, 1024 + 64
+    rng = np.random.default_rng(13)
+    suffixes = [int(x) for x in rng.integers(0, 200, size=24)]
+    s, pblocks = len(suffixes), prefix_len // bs
+    cache, k_host, v_host, _ = cascade_case(dtype, hkv, d, bs, prefix_len, suffixes, 14)
+    scale = 1.0 / math.sqrt(d)
+    prefix_ids = cache.d_tables[0, :pblocks].contiguous()
+    suffix_tables = cache.d_tables[:, pblocks:]
+    suffix_lens = (cache.d_lens - prefix_len).contiguous()
+    q_hosts = [workloads.randn((s, hq, d), dtype, 30 + i) for i in range(2)]
+    qs = [q.cuda() for q in q_hosts]
+    torch.cuda.synchronize()
+    outs = [[], []]
+    errors = []
+
+    def worker(i):
+        try:
+            stream = torch.cuda.Stream()
+            ws = None
+            with torch.cuda.stream(stream):
+                for _ in range(20):
+                    out = torch.full((s, hq, d), float("nan"), dtype=TORCH[dtype], device="cuda")
+                    ws = pa.pa_decode_attention_shared_prefix(qs[i], cache.k_cache, cache.v_cache, prefix_ids,
+                                                              prefix_len, suffix_tables, suffix_lens, scale, out,
+                                                              partition_size=256, workspace=ws, stream=stream)
+                    outs[i].append(out)
+            stream.synchronize()
+        except Exception as e:      # reported on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    assert pa.pa_device_error() == 0
+    for i in range(2):
+        ref = oracle_decode(q_hosts[i].double().numpy(), AsF64(k_host), AsF64(v_host),
+                            [list(r) for r in cache.tables], [int(x) for x in cache.lens], scale)
+        first = outs[i][0].float().cpu().numpy()
+        assert_close(first, ref, dtype, "thread %d" % i)
+        for j, o in enumerate(outs[i][1:]):
+            assert np.array_equal(o.float().cpu().numpy(), first), (i, j)
+
+
 def test_zero_prefix_is_the_plain_call(pa):
     gpu, ref, plain = run_cascade(pa, "bf16", 8, 2, 128, 16, 0, [5, 40], 0, seed=7)
     assert_close(gpu, ref, "bf16", "no prefix")
