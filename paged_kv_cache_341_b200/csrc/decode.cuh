@@ -1386,16 +1386,22 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
     // Shared-prefix slots, most of them empty (m = -inf, left so by the
     // prefix kernel's segments): the (m, l) sweep first, then only the rows
     // of slots that hold tokens, found by a ballot.  Every warp of the head
-    // computes M and L in one sweep as above.
-    for (int p = lane; p < np; p += 32) {
-      const float2 ml = prm.part_ml[base + p];
+    // computes M and L in one sweep as above; the pairs of the first 64 slots
+    // stay in registers, so the rows of all their non-empty slots are loaded
+    // in one round after the sweep.
+    const float2 ml0 = lane < np ? prm.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
+    const float2 ml1 = lane + 32 < np ? prm.part_ml[base + lane + 32] : make_float2(-INFINITY, 0.f);
+    auto take = [&](float2 ml) {
       if (ml.x > mx) {
         lsum = lsum * exp2_approx(mx - ml.x) + ml.y;     // exp2(-inf) = 0 on the first pair
         mx = ml.x;
       } else if (ml.x != -INFINITY) {
         lsum += ml.y * exp2_approx(ml.x - mx);
       }
-    }
+    };
+    take(ml0);
+    take(ml1);
+    for (int p = lane + 64; p < np; p += 32) take(prm.part_ml[base + p]);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {
       const float mo = __shfl_xor_sync(0xffffffffu, mx, off);
@@ -1411,18 +1417,54 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
     // (m, l) pairs and its row is never read.
     const unsigned share = wph == 1 ? 0xffffffffu
                                     : (wph == 2 ? 0x55555555u : (wph == 4 ? 0x11111111u : 0x01010101u)) << sub;
-    for (int p0 = 0; p0 < np; p0 += 32) {
+    // slots 0..63: bit b of todo[c] is slot 32 c + b
+    unsigned todo[2] = {__ballot_sync(0xffffffffu, ml0.x != -INFINITY) & share,
+                        __ballot_sync(0xffffffffu, ml1.x != -INFINITY) & share};
+    while (todo[0] | todo[1]) {
+      int pk[4];
+      int n = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = todo[0] ? 0 : 1;
+        pk[u] = -1;
+        if (todo[c]) {
+          pk[u] = 32 * c + __ffs(todo[c]) - 1;
+          todo[c] &= todo[c] - 1;
+          ++n;
+        }
+      }
+      float2 v[4][PER / 2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u < n) {
+          const float2* src = reinterpret_cast<const float2*>(prm.part_acc + (base + pk[u]) * D + lane * PER);
+#pragma unroll
+          for (int e = 0; e < PER / 2; ++e) v[u][e] = src[e];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u < n) {
+          const float m0 = __shfl_sync(0xffffffffu, ml0.x, pk[u] & 31);
+          const float m1 = __shfl_sync(0xffffffffu, ml1.x, pk[u] & 31);
+          const float wu = exp2_approx((pk[u] < 32 ? m0 : m1) - mx);
+#pragma unroll
+          for (int e = 0; e < PER / 2; ++e) ffma2(o[e], make_float2(wu, wu), v[u][e]);
+        }
+      }
+    }
+    for (int p0 = 64; p0 < np; p0 += 32) {
       const int pl = p0 + lane;
       const float ml_x = pl < np ? prm.part_ml[base + pl].x : -INFINITY;
-      unsigned todo = __ballot_sync(0xffffffffu, ml_x != -INFINITY) & share;
-      while (todo) {
+      unsigned rest = __ballot_sync(0xffffffffu, ml_x != -INFINITY) & share;
+      while (rest) {
         int pk[4];
         int n = 0;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          pk[u] = todo ? __ffs(todo) - 1 : -1;
-          if (todo) {
-            todo &= todo - 1;
+          pk[u] = rest ? __ffs(rest) - 1 : -1;
+          if (rest) {
+            rest &= rest - 1;
             ++n;
           }
         }
