@@ -126,6 +126,15 @@ def test_many_sequences_and_row_tiles(pa, prefix_path, nseq):
     assert_close(gpu, ref, "bf16", "%d sequences" % nseq)
 
 
+def test_prefix_of_more_than_64_slices(pa, prefix_path):
+    # 33,280 prefix tokens = 65 slices of 512 plus the suffix partitions: the
+    # merge reads the (m, l) pairs of slots 64 and up in a second sweep
+    gpu, ref, plain = run_cascade(pa, "bf16", 8, 2, 128, 16, 33280, [0, 5, 300, 77], 256, seed=9)
+    check_launched(pa, prefix_path, 128)
+    assert_close(gpu, ref, "bf16", "%s, 65 prefix slices" % prefix_path)
+    assert_close(gpu, plain.astype(np.float64), "bf16", "%s, 65 prefix slices vs plain call" % prefix_path)
+
+
 def test_large_scores_rescale_in_tensor_memory(pa, prefix_path):
     # queries scaled up so the running maximum moves by more than 2^8 between
     # tiles: the tcgen05 kernel rescales O inside tensor memory
