@@ -43,3 +43,21 @@ def test_reference_config_matches_the_reserved_lengths():
     lens = sc.cache.lens[sc.rows]
     assert cfg["mean_context"] == round(float(np.mean(lens)), 1)
     assert cfg["max_context"] == int(np.max(lens))
+
+
+def test_call_label_names_the_kernels_that_run(monkeypatch):
+    # the roofline's kernel label follows the launch rules: the one-warp
+    # planner for batches of up to 32 sequences, the SM-pair prefix kernel
+    # unless PA_PREFIX_PATH picks another
+    monkeypatch.delenv("PA_PREFIX_PATH", raising=False)
+    monkeypatch.delenv("PA_DECODE_PATH", raising=False)
+    w70 = workloads.WORKLOADS["long_70b_gqa"]
+    w3 = workloads.WORKLOADS["llama3_8b_gqa"]
+    wsp = workloads.WORKLOADS["shared_prefix"]
+    assert "plan_small_kernel + decode_mma_kernel" in bench.call_label(False, w70, 8, 300, "measured")
+    assert "(plan_kernel + decode_mma_kernel" in bench.call_label(False, w3, 256, 300, "measured")
+    assert "prefix_pair_kernel + plan_kernel" in bench.call_label(True, wsp, 200, 300, "measured")
+    monkeypatch.setenv("PA_PREFIX_PATH", "umma")
+    assert "prefix_umma_kernel" in bench.call_label(True, wsp, 200, 300, "measured")
+    monkeypatch.setenv("PA_PREFIX_PATH", "mma")
+    assert "prefix_attention_kernel" in bench.call_label(True, wsp, 200, 300, "measured")
