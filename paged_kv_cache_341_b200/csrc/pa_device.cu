@@ -321,18 +321,19 @@ struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
   CUcontext ctx = nullptr;
-  std::mutex mu;              // one call's fork, launches and join at a time
+  std::mutex mu;              // its creation, and one call's fork, launches and join at a time
 };
 
-pa_status side_stream(SideStream** out) {
-  static std::mutex mu;
+// The current device's side stream, returned with its mutex held in *hold
+// (creation, or re-creation for another context, happens under it too).
+pa_status side_stream(SideStream** out, std::unique_lock<std::mutex>* hold) {
   static SideStream cache[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev >= 64) return pa::fail(PA_ERR_UNSUPPORTED, "shared prefix: device index above 63");
-  std::lock_guard<std::mutex> lock(mu);
   SideStream& s = cache[dev];
+  std::unique_lock<std::mutex> lock(s.mu);
   const CUcontext ctx = current_context();
   if (!s.stream || (ctx && s.ctx && ctx != s.ctx)) {
     // (the handles of a context that is gone are dropped, not destroyed)
@@ -349,6 +350,7 @@ pa_status side_stream(SideStream** out) {
     s.ctx = current_context();
   }
   *out = &s;
+  *hold = std::move(lock);
   return PA_OK;
 }
 
@@ -607,9 +609,9 @@ pa_status pa_decode_attention_shared_prefix(const void* q, const void* k_cache, 
   // after both (the side stream joins before it).  The two halves share no
   // data until the merge, so they may run in either order or together.
   SideStream* ss = nullptr;
-  pa_status st = side_stream(&ss);
+  std::unique_lock<std::mutex> lock;
+  pa_status st = side_stream(&ss, &lock);
   if (st != PA_OK) return st;
-  std::lock_guard<std::mutex> lock(ss->mu);
   cudaError_t e = cudaEventRecord(ss->fork, a.stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
   if (e != cudaSuccess) return cuda_fail(e, "shared prefix: fork to the side stream");
